@@ -1,0 +1,254 @@
+/*
+ * qvae_oracle.c -- plain CPU definition of the W8A8 CausalConv3d layer.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, the smoke check and
+ * the benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA path and must stay slow and
+ * obviously correct: every function is the definition written out, with no
+ * blocking, fusion or reordering.
+ *
+ * What it follows (ComfyUI-Qwen-VAE-Triton v0.2.0 release note, sd114.wiki):
+ *   - section "three presets": weights are symmetric INT8 with one scale per
+ *     output channel; activations are dynamic symmetric INT8; products are
+ *     INT8 x INT8 accumulated in INT32, rescaled in FP32, and the output keeps
+ *     the activation's original precision (bf16 here);
+ *   - same section, "fixed internal parameters": activation and weight clip
+ *     ratios are 1.0, channels_last layout;
+ *   - opening paragraph: the layer is a CausalConv3d (implicit-GEMM lowering
+ *     is only how the kernel evaluates it; the result is the plain sum below).
+ * Readings where the page is silent (each listed in the design doc):
+ *   - activation scale is per tensor; scale = absmax / 127 (IEEE fp32 divide);
+ *   - code = clamp(rint(v / scale), -127, 127), rint = round half to even,
+ *     v / scale an IEEE fp32 divide; absmax == 0 gives scale 0 and all codes 0;
+ *   - causal padding is two leading zero frames (kernel slice kt = 2 meets
+ *     frame t, kt = 0 meets frame t - 2), spatial padding 1, stride 1, 3x3x3;
+ *   - epilogue: y = float(acc) * (s_a * s_w[co]), then y + float(bias[co]) as
+ *     a separate add (no fused multiply-add), then bf16 round-to-nearest-even.
+ *
+ * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -shared -fPIC (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_NONFINITE 1
+#define ORC_ERR_OVERFLOW 2
+#define ORC_ERR_ARG 3
+
+/* bf16 is the upper half of an IEEE binary32: widening is exact. */
+static float bf16_bits_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even (inputs are finite). */
+static uint16_t float_to_bf16_bits(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) /* NaN: keep it quiet */
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep_lsb = (u >> 16) & 1u;
+    u += 0x7fffu + keep_lsb;
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_bits(f); }
+
+/* One INT8 code: clamp(rint(v / s), -127, 127); s == 0 maps to code 0. */
+static int8_t quantize_one(float v, float s)
+{
+    if (s == 0.0f)
+        return 0;
+    float r = rintf(v / s);
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/*
+ * Weight quantisation, per output channel.
+ * w: bf16 bits, PyTorch Conv3d weight [Cout][Cin][3][3][3] (contiguous).
+ * qw: INT8 codes in the same layout.  s_w: [Cout] fp32 scales.
+ */
+int oracle_quantize_weights(const uint16_t *w, int32_t Cout, int32_t Cin,
+                            int8_t *qw, float *s_w)
+{
+    if (Cout <= 0 || Cin <= 0) return ORC_ERR_ARG;
+    const int64_t per_co = (int64_t)Cin * 27;
+    for (int32_t co = 0; co < Cout; ++co) {
+        const uint16_t *wc = w + (int64_t)co * per_co;
+        float amax = 0.0f;
+        for (int64_t i = 0; i < per_co; ++i) {
+            float v = bf16_bits_to_float(wc[i]);
+            if (!isfinite(v)) return ORC_ERR_NONFINITE;
+            float a = fabsf(v);
+            if (a > amax) amax = a;
+        }
+        amax = amax * 1.0f;          /* weight clip ratio 1.0 */
+        float s = amax / 127.0f;
+        s_w[co] = s;
+        for (int64_t i = 0; i < per_co; ++i)
+            qw[(int64_t)co * per_co + i] = quantize_one(bf16_bits_to_float(wc[i]), s);
+    }
+    return ORC_OK;
+}
+
+/* Per-tensor absmax of a bf16 tensor (any layout; every element counts). */
+int oracle_act_absmax(const uint16_t *x, int64_t numel, float *amax_out)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < numel; ++i) {
+        float v = bf16_bits_to_float(x[i]);
+        if (!isfinite(v)) return ORC_ERR_NONFINITE;
+        float a = fabsf(v);
+        if (a > amax) amax = a;
+    }
+    *amax_out = amax;
+    return ORC_OK;
+}
+
+/*
+ * Dynamic per-tensor activation quantisation.
+ * x: bf16 bits, numel elements.  qx: INT8 codes, same order.  s_a: scale.
+ */
+int oracle_act_quant(const uint16_t *x, int64_t numel, int8_t *qx, float *s_a)
+{
+    float amax;
+    int rc = oracle_act_absmax(x, numel, &amax);
+    if (rc != ORC_OK) return rc;
+    amax = amax * 1.0f;              /* activation clip ratio 1.0 */
+    float s = amax / 127.0f;
+    *s_a = s;
+    for (int64_t i = 0; i < numel; ++i)
+        qx[i] = quantize_one(bf16_bits_to_float(x[i]), s);
+    return ORC_OK;
+}
+
+/*
+ * The causal 3x3x3 convolution of the codes, accumulated exactly.
+ * One output point (n, t, h, w, co):
+ *   acc = sum over kt, kh, kw in {0,1,2} and ci of
+ *         qx[n, t + kt - 2, h + kh - 1, w + kw - 1, ci] * qw[co, ci, kt, kh, kw]
+ * where any input index outside the tensor contributes zero (two leading
+ * zero frames in time, one zero pixel on each spatial side).
+ * qx: [N][T][H][W][Cin] (channels_last); qw: [Cout][Cin][3][3][3].
+ */
+static int conv_point(const int8_t *qx, const int8_t *qw, int64_t T, int64_t H,
+                      int64_t W, int32_t Cin, int64_t n, int64_t t, int64_t h,
+                      int64_t w, int32_t co, int32_t *out)
+{
+    int64_t acc = 0;
+    for (int kt = 0; kt < 3; ++kt) {
+        int64_t ti = t + kt - 2;
+        if (ti < 0 || ti >= T) continue;
+        for (int kh = 0; kh < 3; ++kh) {
+            int64_t hi = h + kh - 1;
+            if (hi < 0 || hi >= H) continue;
+            for (int kw = 0; kw < 3; ++kw) {
+                int64_t wi = w + kw - 1;
+                if (wi < 0 || wi >= W) continue;
+                const int8_t *xp = qx + ((((n * T + ti) * H + hi) * W + wi) * Cin);
+                for (int32_t ci = 0; ci < Cin; ++ci) {
+                    int64_t widx = ((((int64_t)co * Cin + ci) * 3 + kt) * 3 + kh) * 3 + kw;
+                    acc += (int64_t)xp[ci] * (int64_t)qw[widx];
+                }
+            }
+        }
+    }
+    if (acc > INT32_MAX || acc < INT32_MIN) return ORC_ERR_OVERFLOW;
+    *out = (int32_t)acc;
+    return ORC_OK;
+}
+
+/* Every output point; acc: [N][T][H][W][Cout]. */
+int oracle_conv_acc(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
+                    int64_t H, int64_t W, int32_t Cin, int32_t Cout, int32_t *acc)
+{
+    if (N <= 0 || T <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0) return ORC_ERR_ARG;
+    int rc_all = ORC_OK;
+    const int64_t rows = N * T * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t n = r / (T * H), t = (r / H) % T, h = r % H;
+        for (int64_t w = 0; w < W; ++w)
+            for (int32_t co = 0; co < Cout; ++co) {
+                int32_t v = 0;
+                int rc = conv_point(qx, qw, T, H, W, Cin, n, t, h, w, co, &v);
+                if (rc != ORC_OK) {
+#pragma omp atomic write
+                    rc_all = rc;
+                }
+                acc[(((n * T + t) * H + h) * W + w) * Cout + co] = v;
+            }
+    }
+    return rc_all;
+}
+
+/* Selected output pixels only; pts: [npts][4] = (n, t, h, w); acc: [npts][Cout]. */
+int oracle_conv_acc_points(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
+                           int64_t H, int64_t W, int32_t Cin, int32_t Cout,
+                           const int64_t *pts, int64_t npts, int32_t *acc)
+{
+    int rc_all = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npts; ++p) {
+        const int64_t *q = pts + 4 * p;
+        int bad = q[0] < 0 || q[0] >= N || q[1] < 0 || q[1] >= T || q[2] < 0 ||
+                  q[2] >= H || q[3] < 0 || q[3] >= W;
+        for (int32_t co = 0; co < Cout; ++co) {
+            int32_t v = 0;
+            int rc = bad ? ORC_ERR_ARG
+                         : conv_point(qx, qw, T, H, W, Cin, q[0], q[1], q[2], q[3], co, &v);
+            if (rc != ORC_OK) {
+#pragma omp atomic write
+                rc_all = rc;
+            }
+            acc[p * Cout + co] = v;
+        }
+    }
+    return rc_all;
+}
+
+/*
+ * FP32 rescale, bias, cast back to bf16.
+ * acc: [M][Cout]; s_w: [Cout]; bias: bf16 bits [Cout] or NULL (zero bias).
+ */
+void oracle_epilogue(const int32_t *acc, int64_t M, int32_t Cout, float s_a,
+                     const float *s_w, const uint16_t *bias, uint16_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int32_t co = 0; co < Cout; ++co) {
+            float scale = s_a * s_w[co];
+            float y = (float)acc[m * Cout + co] * scale;
+            float b = bias ? bf16_bits_to_float(bias[co]) : 0.0f;
+            y = y + b;
+            out[m * Cout + co] = float_to_bf16_bits(y);
+        }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
