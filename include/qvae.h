@@ -1,0 +1,207 @@
+/*
+ * qvae.h -- C ABI of libqvae: the W8A8 CausalConv3d layer of the Qwen-Image /
+ * Wan VAE decoder on NVIDIA B200 (sm_100a).
+ *
+ * The method (ComfyUI-Qwen-VAE-Triton v0.2.0 release note, sd114.wiki):
+ *   - opening paragraph: an implicit-GEMM W8A8 kernel for the decoder's
+ *     CausalConv3d layers;
+ *   - section on the three presets: weights are symmetric INT8 with one scale
+ *     per output channel, activations dynamic symmetric INT8, INT8 x INT8
+ *     products accumulated in INT32, rescaled in FP32, and the output keeps
+ *     the activation's precision; clip ratios 1.0; channels_last; a failing
+ *     quantised layer falls back to the native one (here: every call returns
+ *     a status and never aborts, the caller decides the fallback);
+ *   - the Aggressive preset quantises 26 of 28 layers and leaves 2 in native
+ *     precision (here: the `quantized` flag of qvae_layer).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned.  bf16 tensors are channels_last: [N][T][H][W][C], C fastest.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work; nothing synchronises the host, and scales stay on the
+ *     device.  The library allocates no device memory.
+ *   - Return value: QVAE_OK or a qvae_status code.  Argument errors are
+ *     detected before anything is launched.  A device-side wait that ran out
+ *     of time is reported later by qvae_get_error().
+ *   - Layer geometry is fixed: 3x3x3 kernel, stride 1, causal temporal
+ *     padding of 2 leading zero frames, spatial padding 1 ("same" size).
+ */
+#ifndef QVAE_H
+#define QVAE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The library is built with hidden visibility; everything declared here is exported. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef enum qvae_status {
+  QVAE_OK = 0,
+  QVAE_ERR_ARG = 1,      /* null pointer, negative size, bad workspace */
+  QVAE_ERR_SHAPE = 2,    /* Cin or Cout not a multiple of 32, or sizes out of range */
+  QVAE_ERR_ALIGN = 3,    /* a pointer is not 16-byte aligned */
+  QVAE_ERR_CUDA = 4,     /* a CUDA call or kernel launch failed */
+  QVAE_ERR_TIMEOUT = 5,  /* a device-side pipeline wait ran out of time */
+  QVAE_ERR_UNSUPPORTED = 6
+} qvae_status;
+
+/* Shape of one CausalConv3d layer; input and output have the same N, T, H, W. */
+typedef struct qvae_shape {
+  int64_t N, T, H, W;
+  int32_t Cin, Cout;
+} qvae_shape;
+
+/* Human-readable text of a status code (static storage). */
+const char* qvae_status_string(int status);
+
+/* Text of the last CUDA error seen by this library on the calling thread. */
+const char* qvae_last_error_message(void);
+
+/* ------------------------------------------------------------- weights -- */
+
+/* Bytes of the packed weight buffer for a layer:
+ * 27 taps x ceil(Cin/128) chunks x Cout rows x 128 bytes. */
+size_t qvae_packed_weight_bytes(int32_t Cin, int32_t Cout);
+
+/*
+ * One-time weight quantisation and repack (release note, three presets:
+ * "weights symmetric INT8, one scale per output channel", clip ratio 1.0).
+ *   w_bf16     [Cout][Cin][3][3][3] bf16, the PyTorch Conv3d weight layout.
+ *   wq_packed  qvae_packed_weight_bytes(Cin, Cout) bytes, written: INT8 codes
+ *              in the convolution's consumption order, [tap][chunk][Cout][128]
+ *              with tap = (kt*3 + kh)*3 + kw, each 128-byte row holding 128
+ *              input channels in the tensor cores' 128-byte swizzle (16-byte
+ *              group g at position g ^ (co % 8)), zeros beyond Cin.
+ *   w_scale    [Cout] fp32, written: absmax(w[co]) / 127.
+ *   wq_plain   optional (NULL to skip): [Cout][27][Cin] codes, tap-major.
+ * code = clamp(rint(w / w_scale[co]), -127, 127), IEEE divide, half to even;
+ * an all-zero output channel gets scale 0 and zero codes.
+ * Needs Cin % 32 == 0 and Cout % 32 == 0.
+ */
+int qvae_quantize_weights(int32_t Cin, int32_t Cout, const void* w_bf16, int8_t* wq_packed,
+                          float* w_scale, int8_t* wq_plain, void* stream);
+
+/* ---------------------------------------------------------- activations -- */
+
+/* Workspace bytes qvae_act_absmax_quant needs (partial maxima); at most 16 KiB. */
+size_t qvae_act_workspace_bytes(int64_t numel);
+
+/*
+ * Dynamic per-tensor activation quantisation (release note, three presets:
+ * "activations dynamic symmetric INT8", clip ratio 1.0).
+ *   x_bf16     numel bf16 values (any layout; every element counts).
+ *   xq         numel INT8 codes, written in the same order.
+ *   x_scale    one fp32 on the device, written: absmax(x) / 127.
+ *   workspace  qvae_act_workspace_bytes(numel) bytes of scratch.
+ * code = clamp(rint(x / x_scale), -127, 127) with the IEEE divide's result,
+ * half to even; an all-zero tensor gets scale 0 and zero codes.  Inputs must
+ * be finite.  numel == 0 writes scale 0 and nothing else.
+ */
+int qvae_act_absmax_quant(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------- convolution -- */
+
+/*
+ * The W8A8 causal 3x3x3 convolution (release note: opening paragraph and the
+ * three-presets section):
+ *   acc[n,t,h,w,co] = sum over kt,kh,kw,ci of
+ *                     xq[n, t+kt-2, h+kh-1, w+kw-1, ci] * wq[co, ci, kt, kh, kw]
+ *                     (zero outside the tensor), exact in INT32;
+ *   out[n,t,h,w,co] = bf16_rne( float(acc) * (x_scale * w_scale[co]) + bias[co] ).
+ *   xq         [N][T][H][W][Cin] INT8 codes (from qvae_act_absmax_quant).
+ *   x_scale    device fp32 scalar (from qvae_act_absmax_quant).
+ *   wq_packed, w_scale   from qvae_quantize_weights.
+ *   bias_bf16  [Cout] bf16, or NULL for no bias.
+ *   out_bf16   [N][T][H][W][Cout] bf16, written.
+ * Needs Cin % 32 == 0, Cout % 32 == 0; sizes with N*T*H*W == 0 do nothing.
+ */
+int qvae_causal_conv3d_w8a8(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
+                            const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
+                            void* out_bf16, void* stream);
+
+/* Same convolution, writing the raw INT32 accumulators acc [N][T][H][W][Cout]
+ * instead of the bf16 output (for exact checking). */
+int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
+                                  const int8_t* wq_packed, int32_t* acc, void* stream);
+
+/* ---------------------------------------------------------- layer chain -- */
+
+/*
+ * One decoder layer for qvae_decode_layers.  quantized == 0 marks a layer
+ * kept in native precision (the release note's Aggressive preset keeps 2 of
+ * 28); the library skips it and the caller runs it.
+ */
+typedef struct qvae_layer {
+  qvae_shape shape;
+  int32_t quantized;
+  int32_t reserved;          /* set to 0 */
+  const void* x;             /* bf16 [N][T][H][W][Cin] */
+  void* out;                 /* bf16 [N][T][H][W][Cout] */
+  const int8_t* wq_packed;   /* from qvae_quantize_weights */
+  const float* w_scale;      /* [Cout] */
+  const void* bias;          /* bf16 [Cout] or NULL */
+} qvae_layer;
+
+/* Workspace bytes qvae_decode_layers needs for these layers. */
+size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
+
+/*
+ * For each layer with quantized != 0, in order on one stream: activation
+ * absmax + quantise into the workspace, then the convolution into `out`.
+ * All layers are validated before anything is launched.
+ */
+int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* -------------------------------------------------------------- control -- */
+
+/*
+ * Waits for `stream`, then returns and clears the device error word:
+ * QVAE_OK, QVAE_ERR_TIMEOUT (a pipeline wait inside a kernel gave up; the
+ * results of that call are invalid), or QVAE_ERR_CUDA if the wait failed.
+ */
+int qvae_get_error(void* stream);
+
+/*
+ * Time limit of every device-side pipeline wait, in nanoseconds (default
+ * 2e9).  A wait past it makes the kernel record QVAE_ERR_TIMEOUT, wait
+ * (bounded) for its own copies in flight, free its tensor memory and return.
+ */
+int qvae_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * Launches a kernel whose only wait can never be satisfied, with the given
+ * limit: the wait must give up and qvae_get_error() must then report
+ * QVAE_ERR_TIMEOUT.  Exercises the timeout path without faulting the GPU.
+ */
+int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
+ * Convolution tiling override for tuning and tests (process-wide, not
+ * thread-safe).  BW: tile width in pixels (8, 16, 32, 64 or 128; tile height
+ * is 128/BW rows), MS: 128-pixel sub-tiles stacked per CTA tile (1 or 2),
+ * NT: output channels per CTA tile (a multiple of 32 dividing Cout, <= 256),
+ * SA / SB: activation / weight pipeline stages (<= 8).  Zero = automatic.
+ */
+int qvae_set_conv_tiling(int32_t BW, int32_t MS, int32_t NT, int32_t SA, int32_t SB);
+
+/* The tiling the next convolution of this shape would use:
+ * out[0..6] = BW, BH, MS, NT, SA, SB, number of CTA tiles. */
+int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QVAE_H */

@@ -1,0 +1,117 @@
+"""The C ABI library: it loads, exports every declared symbol, and rejects bad
+arguments before touching the GPU (no compute calls here; runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from video_vae_decode_b200 import qvae
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qvae.h")
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced
+FAKE_ODD = ctypes.c_void_p(0x10008)      # misaligned
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qvae_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(qvae.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = qvae.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = qvae.lib()
+    for code in range(7):
+        assert L.qvae_status_string(code)
+    assert L.qvae_status_string(99) == b"unknown status"
+
+
+def test_packed_weight_bytes():
+    assert qvae.qvae_packed_weight_bytes(384, 384) == 27 * 3 * 384 * 128
+    assert qvae.qvae_packed_weight_bytes(96, 96) == 27 * 1 * 96 * 128
+    assert qvae.qvae_packed_weight_bytes(192, 96) == 27 * 2 * 96 * 128
+    assert qvae.qvae_packed_weight_bytes(0, 96) == 0
+
+
+def conv(shape, xq=FAKE, xs=FAKE, wq=FAKE, ws=FAKE, b=None, out=FAKE):
+    return qvae.lib().qvae_causal_conv3d_w8a8(ctypes.byref(shape), xq, xs, wq, ws, b, out, None)
+
+
+def test_conv_argument_checks():
+    ok = qvae.make_shape(1, 1, 8, 8, 64, 64)
+    assert conv(qvae.make_shape(1, 1, 8, 8, 48, 64)) == qvae.QVAE_ERR_SHAPE
+    assert conv(qvae.make_shape(1, 1, 8, 8, 64, 40)) == qvae.QVAE_ERR_SHAPE
+    assert conv(qvae.make_shape(1, 1, 8, 8, 16, 64)) == qvae.QVAE_ERR_SHAPE
+    assert conv(qvae.make_shape(-1, 1, 8, 8, 64, 64)) == qvae.QVAE_ERR_ARG
+    assert conv(ok, xq=None) == qvae.QVAE_ERR_ARG
+    assert conv(ok, xs=None) == qvae.QVAE_ERR_ARG
+    assert conv(ok, out=FAKE_ODD) == qvae.QVAE_ERR_ALIGN
+    assert conv(ok, xq=FAKE_ODD) == qvae.QVAE_ERR_ALIGN
+    assert conv(qvae.make_shape(1, 0, 8, 8, 64, 64), xq=None) == qvae.QVAE_OK   # empty: no-op
+    L = qvae.lib()
+    assert L.qvae_causal_conv3d_w8a8(None, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_causal_conv3d_w8a8_acc32(ctypes.byref(ok), FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+
+
+def test_act_and_weight_argument_checks():
+    L = qvae.lib()
+    ws = qvae.qvae_act_workspace_bytes(1000)
+    assert L.qvae_act_absmax_quant(FAKE, -1, FAKE, FAKE, FAKE, ws, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_absmax_quant(FAKE, 100, FAKE, FAKE, FAKE, 16, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_absmax_quant(FAKE_ODD, 100, FAKE, FAKE, FAKE, ws, None) == qvae.QVAE_ERR_ALIGN
+    assert L.qvae_act_absmax_quant(FAKE, 100, FAKE, None, FAKE, ws, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_quantize_weights(48, 64, FAKE, FAKE, FAKE, None, None) == qvae.QVAE_ERR_SHAPE
+    assert L.qvae_quantize_weights(64, 64, None, FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_quantize_weights(64, 64, FAKE, FAKE_ODD, FAKE, None, None) == qvae.QVAE_ERR_ALIGN
+
+
+def test_decode_layers_validates_everything_first():
+    L = qvae.lib()
+    arr = (qvae.qvae_layer * 2)()
+    for i in range(2):
+        arr[i].shape = qvae.make_shape(1, 1, 8, 8, 64, 64)
+        arr[i].quantized = 1
+        arr[i].x = arr[i].out = arr[i].wq_packed = arr[i].w_scale = 0x10000
+    arr[1].shape = qvae.make_shape(1, 1, 8, 8, 48, 64)
+    need = L.qvae_decode_workspace_bytes(arr, 2)
+    assert L.qvae_decode_layers(arr, 2, FAKE, need, None) == qvae.QVAE_ERR_SHAPE
+    arr[1].quantized = 0                                   # pass-through layers are not checked
+    need = L.qvae_decode_workspace_bytes(arr, 2)
+    assert need >= 8 * 8 * 64
+    assert L.qvae_decode_layers(arr, 2, FAKE, need - 1, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_decode_layers(arr, -1, FAKE, need, None) == qvae.QVAE_ERR_ARG
+
+
+def test_tiling_choice_is_valid():
+    for (N, T, H, W, Cin, Cout) in [(1, 1, 128, 128, 384, 384), (1, 1, 64, 64, 96, 96),
+                                    (1, 1, 105, 157, 384, 384), (1, 8, 240, 416, 192, 192),
+                                    (1, 1, 1024, 1024, 192, 96), (1, 1, 840, 1256, 96, 96)]:
+        t = qvae.qvae_get_conv_tiling(N, T, H, W, Cin, Cout)
+        assert t["BW"] * t["BH"] == 128 and t["MS"] in (1, 2)
+        assert Cout % t["NT"] == 0 and t["NT"] % 32 == 0 and t["NT"] <= 256
+        assert 1 <= t["SA"] <= 8 and 1 <= t["SB"] <= 8
+        rows = t["MS"] * t["BH"]
+        tiles = N * T * -(-H // rows) * -(-W // t["BW"]) * (Cout // t["NT"])
+        assert t["tiles"] == tiles
+    qvae.qvae_set_conv_tiling(BW=32, MS=1, NT=64, SA=2, SB=3)
+    try:
+        t = qvae.qvae_get_conv_tiling(1, 1, 100, 100, 128, 128)
+        assert (t["BW"], t["BH"], t["MS"], t["NT"], t["SA"], t["SB"]) == (32, 4, 1, 64, 2, 3)
+    finally:
+        qvae.qvae_set_conv_tiling()
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(BW=24)
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(NT=48)

@@ -1,0 +1,228 @@
+// quant.cuh -- INT8 quantisation kernels.
+//
+// Scheme (ComfyUI-Qwen-VAE-Triton v0.2.0 release note, "three presets"):
+// weights are symmetric INT8 with one scale per output channel, activations
+// are dynamic symmetric INT8 (one scale per tensor), clip ratio 1.0 for both.
+// scale = absmax / 127 and code = clamp(rint(v / scale), -127, 127) with an
+// IEEE round-to-nearest divide and round-half-to-even; absmax == 0 gives
+// scale 0 and all-zero codes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qvae {
+
+// |bf16| ordering equals the unsigned ordering of its low 15 bits (finite
+// inputs), so absmax is taken on integers and widened once at the end.
+__device__ __forceinline__ uint32_t abs_bits_max2(uint32_t m, uint32_t word) {
+  const uint32_t lo = word & 0x7FFFu, hi = (word >> 16) & 0x7FFFu;
+  return max(m, max(lo, hi));
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// Rounded quotient v / s to the nearest integer (ties to even), clamped to
+// [-127, 127], returned as the low byte of a float's bit pattern.
+//
+// The quotient is the IEEE round-to-nearest v / s.  It is computed from
+// r = RN(1 / s) with one multiply and one remainder correction (Markstein's
+// correctly rounded division: q0 = RN(v r), e = fma(-q0, s, v) exactly,
+// q = fma(e, r, q0)); the activation tests check it code-for-code against
+// the plain divide over every bf16 input for many scales.  Rounding to an
+// integer adds 1.5 * 2^23: the sum lies in [2^23, 2^24) where the spacing is
+// 1, so the IEEE add rounds half to even, and the low mantissa byte is the
+// two's-complement code.
+struct Quantizer {
+  float s, r;
+  bool exact;  // plain divide (tiny scales whose reciprocal overflows)
+  __device__ __forceinline__ uint32_t code_byte(float v) const {
+    float q;
+    if (exact) {
+      q = __fdiv_rn(v, s);
+    } else {
+      const float q0 = __fmul_rn(v, r);
+      const float e = __fmaf_rn(-q0, s, v);
+      q = __fmaf_rn(e, r, q0);
+    }
+    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(q, 12582912.0f)) & 0xFFu;
+  }
+};
+
+__device__ __forceinline__ Quantizer make_quantizer(float s) {
+  Quantizer z;
+  z.s = s;
+  z.r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+  z.exact = !(s >= 0x1p-100f);
+  return z;
+}
+
+// Four bf16 (two 32-bit words) -> four packed codes.
+__device__ __forceinline__ uint32_t quant4(const Quantizer& z, uint32_t w0, uint32_t w1) {
+  const uint32_t c0 = z.code_byte(__uint_as_float(w0 << 16));
+  const uint32_t c1 = z.code_byte(__uint_as_float(w0 & 0xFFFF0000u));
+  const uint32_t c2 = z.code_byte(__uint_as_float(w1 << 16));
+  const uint32_t c3 = z.code_byte(__uint_as_float(w1 & 0xFFFF0000u));
+  return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+}
+
+template <int kThreads>
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (warp == 0) {
+    m = (lane < kThreads / 32) ? red[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) red[0] = m;
+  }
+  __syncthreads();
+  const uint32_t r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// ------------------------------------------------------------ activations
+
+constexpr int kActThreads = 256;
+
+// Pass 1: per-block absmax (as 15-bit magnitude codes) of a bf16 tensor.  Plain cached
+// loads: when x fits in L2 the second pass reads it from there.
+// x is 16-byte aligned; nvec = numel / 8 full vectors; block 0 also covers the tail.
+__global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __restrict__ x,
+                                                                  int64_t nvec,
+                                                                  const uint16_t* __restrict__ xs,
+                                                                  int64_t numel,
+                                                                  uint32_t* __restrict__ partial) {
+  __shared__ uint32_t red[kActThreads / 32];
+  uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    const uint4 a = __ldg(x + i), b = __ldg(x + i + stride);
+    const uint4 c = __ldg(x + i + 2 * stride), d = __ldg(x + i + 3 * stride);
+    m0 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m0, a.x), a.y), a.z), a.w);
+    m1 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m1, b.x), b.y), b.z), b.w);
+    m2 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m2, c.x), c.y), c.z), c.w);
+    m3 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m3, d.x), d.y), d.z), d.w);
+  }
+  for (; i < nvec; i += stride) {
+    const uint4 a = __ldg(x + i);
+    m0 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m0, a.x), a.y), a.z), a.w);
+  }
+  if (blockIdx.x == 0) {
+    for (int64_t k = nvec * 8 + threadIdx.x; k < numel; k += kActThreads)
+      m0 = max(m0, static_cast<uint32_t>(xs[k]) & 0x7FFFu);
+  }
+  const uint32_t m = block_max_u32<kActThreads>(max(max(m0, m1), max(m2, m3)), red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+}
+
+// Pass 2: reduce the partial maxima, derive the scale, write INT8 codes.
+// Pairs of 16-byte bf16 vectors become one 16-byte code vector; nvec2 = numel / 16.
+__global__ void __launch_bounds__(kActThreads) act_quant_kernel(
+    const uint4* __restrict__ x, int64_t nvec2, const uint16_t* __restrict__ xs, int64_t numel,
+    const uint32_t* __restrict__ partial, int npartial, uint4* __restrict__ xq,
+    int8_t* __restrict__ xq_bytes, float* __restrict__ x_scale) {
+  __shared__ uint32_t red[kActThreads / 32];
+  uint32_t m = 0;
+  for (int k = threadIdx.x; k < npartial; k += kActThreads) m = max(m, partial[k]);
+  m = block_max_u32<kActThreads>(m, red);
+  const float amax = bf16_bits_to_f32(m) * 1.0f;  // activation clip ratio 1.0
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *x_scale = s;
+  const Quantizer z = make_quantizer(s);
+
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
+  for (; i + stride < nvec2; i += 2 * stride) {
+    const uint4 a0 = __ldcs(x + 2 * i), a1 = __ldcs(x + 2 * i + 1);
+    const uint4 b0 = __ldcs(x + 2 * (i + stride)), b1 = __ldcs(x + 2 * (i + stride) + 1);
+    uint4 qa, qb;
+    if (s == 0.0f) {
+      qa = make_uint4(0, 0, 0, 0);
+      qb = qa;
+    } else {
+      qa = make_uint4(quant4(z, a0.x, a0.y), quant4(z, a0.z, a0.w), quant4(z, a1.x, a1.y),
+                      quant4(z, a1.z, a1.w));
+      qb = make_uint4(quant4(z, b0.x, b0.y), quant4(z, b0.z, b0.w), quant4(z, b1.x, b1.y),
+                      quant4(z, b1.z, b1.w));
+    }
+    xq[i] = qa;
+    xq[i + stride] = qb;
+  }
+  for (; i < nvec2; i += stride) {
+    const uint4 a0 = __ldcs(x + 2 * i), a1 = __ldcs(x + 2 * i + 1);
+    uint4 qa = make_uint4(0, 0, 0, 0);
+    if (s != 0.0f)
+      qa = make_uint4(quant4(z, a0.x, a0.y), quant4(z, a0.z, a0.w), quant4(z, a1.x, a1.y),
+                      quant4(z, a1.z, a1.w));
+    xq[i] = qa;
+  }
+  if (blockIdx.x == 0) {
+    for (int64_t k = nvec2 * 16 + threadIdx.x; k < numel; k += kActThreads) {
+      const uint32_t c = (s == 0.0f) ? 0u : z.code_byte(bf16_bits_to_f32(xs[k]));
+      xq_bytes[k] = static_cast<int8_t>(static_cast<uint8_t>(c));
+    }
+  }
+}
+
+// ---------------------------------------------------------------- weights
+
+constexpr int kWThreads = 256;
+
+// One block per output channel: s_w[co] = absmax(w[co, ...]) / 127.
+// w: bf16 [Cout][Cin][3][3][3] (PyTorch Conv3d layout).
+__global__ void __launch_bounds__(kWThreads) weight_scale_kernel(const uint16_t* __restrict__ w,
+                                                                  int Cin,
+                                                                  float* __restrict__ w_scale) {
+  __shared__ uint32_t red[kWThreads / 32];
+  const int co = blockIdx.x;
+  const int64_t per = static_cast<int64_t>(Cin) * 27;
+  const uint16_t* wc = w + co * per;
+  uint32_t m = 0;
+  for (int64_t k = threadIdx.x; k < per; k += kWThreads) m = max(m, static_cast<uint32_t>(wc[k]) & 0x7FFFu);
+  m = block_max_u32<kWThreads>(m, red);
+  if (threadIdx.x == 0) w_scale[co] = __fdiv_rn(bf16_bits_to_f32(m) * 1.0f, 127.0f);  // clip 1.0
+}
+
+// Codes in the convolution's consumption order.  One thread per packed byte:
+//   packed[tap][chunk][co][128]   tap = (kt * 3 + kh) * 3 + kw, chunk = 128 input channels;
+// inside a 128-byte row the 16-byte group g holds channels chunk*128 + (g ^ (co & 7))*16 + [0,16)
+// (the tensor cores' 128-byte swizzle, so a plain bulk copy lands in MMA layout); channels
+// beyond Cin are zero.  plain (optional): [co][tap][Cin] codes for checking.
+__global__ void weight_pack_kernel(const uint16_t* __restrict__ w, int Cin, int Cout, int nchunks,
+                                   const float* __restrict__ w_scale, int8_t* __restrict__ packed,
+                                   int8_t* __restrict__ plain) {
+  const int64_t total = static_cast<int64_t>(27) * nchunks * Cout * 128;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(idx & 127);
+    int64_t rest = idx >> 7;
+    const int co = static_cast<int>(rest % Cout);
+    rest /= Cout;
+    const int chunk = static_cast<int>(rest % nchunks);
+    const int tap = static_cast<int>(rest / nchunks);
+    const int g = (b >> 4) ^ (co & 7);
+    const int ci = chunk * 128 + g * 16 + (b & 15);
+    uint32_t code = 0;
+    if (ci < Cin) {
+      const int kt = tap / 9, kh = (tap / 3) % 3, kw = tap % 3;
+      const float v = bf16_bits_to_f32(w[((static_cast<int64_t>(co) * Cin + ci) * 3 + kt) * 9 + kh * 3 + kw]);
+      const float s = w_scale[co];
+      if (s != 0.0f) {
+        float q = rintf(__fdiv_rn(v, s));
+        q = fminf(fmaxf(q, -127.0f), 127.0f);
+        code = static_cast<uint32_t>(static_cast<int>(q)) & 0xFFu;
+      }
+      if (plain) plain[(static_cast<int64_t>(co) * 27 + tap) * Cin + ci] = static_cast<int8_t>(code);
+    }
+    packed[idx] = static_cast<int8_t>(static_cast<uint8_t>(code));
+  }
+}
+
+}  // namespace qvae
