@@ -185,15 +185,18 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /*
  * Convolution tiling override for tuning and tests (process-wide, not
- * thread-safe).  BW: tile width in pixels (8, 16, 32, 64 or 128; tile height
- * is 128/BW rows), MS: 128-pixel sub-tiles stacked per CTA tile (1 or 2),
- * NT: output channels per CTA tile (a multiple of 32 dividing Cout, <= 256),
- * SA / SB: activation / weight pipeline stages (<= 8).  Zero = automatic.
+ * thread-safe).  A CTA tile is MS sub-tiles of 128 output pixels (16 image
+ * rows x 8 columns each, stacked vertically) by NT output channels.
+ *   MS    1..4;  NT  a multiple of 32 dividing Cout, <= 256;  MS * NT <= 512
+ *   SA/SB activation / weight pipeline stages (<= 12)
+ *   mode  1 = one CTA per MMA, 2 = CTA pairs (cta_group::2, M = 256 per MMA)
+ * Zero = automatic (a cost model over the shape).  A forced value that
+ * cannot be used for a shape makes the convolution return an error.
  */
-int qvae_set_conv_tiling(int32_t BW, int32_t MS, int32_t NT, int32_t SA, int32_t SB);
+int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode);
 
-/* The tiling the next convolution of this shape would use:
- * out[0..6] = BW, BH, MS, NT, SA, SB, number of CTA tiles. */
+/* The tiling the next convolution of this shape would use: out[0..6] = MS,
+ * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2). */
 int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7);
 
 #if defined(__GNUC__)

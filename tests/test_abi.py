@@ -99,19 +99,24 @@ def test_tiling_choice_is_valid():
                                     (1, 1, 105, 157, 384, 384), (1, 8, 240, 416, 192, 192),
                                     (1, 1, 1024, 1024, 192, 96), (1, 1, 840, 1256, 96, 96)]:
         t = qvae.qvae_get_conv_tiling(N, T, H, W, Cin, Cout)
-        assert t["BW"] * t["BH"] == 128 and t["MS"] in (1, 2)
+        assert 1 <= t["MS"] <= 4 and t["MS"] * t["NT"] <= 512 and t["mode"] in (1, 2)
         assert Cout % t["NT"] == 0 and t["NT"] % 32 == 0 and t["NT"] <= 256
-        assert 1 <= t["SA"] <= 8 and 1 <= t["SB"] <= 8
-        rows = t["MS"] * t["BH"]
-        tiles = N * T * -(-H // rows) * -(-W // t["BW"]) * (Cout // t["NT"])
-        assert t["tiles"] == tiles
-    qvae.qvae_set_conv_tiling(BW=32, MS=1, NT=64, SA=2, SB=3)
+        assert 1 <= t["SA"] <= 12 and 1 <= t["SB"] <= 12
+        assert t["acc_buffers"] == (2 if 2 * t["MS"] * t["NT"] <= 512 else 1)
+        rows = 16 * t["MS"] * t["mode"]
+        tiles = N * T * -(-H // rows) * -(-W // 8) * (Cout // t["NT"])
+        assert t["ctas"] == tiles * t["mode"]
+    qvae.qvae_set_conv_tiling(MS=1, NT=64, SA=2, SB=3, mode=1)
     try:
         t = qvae.qvae_get_conv_tiling(1, 1, 100, 100, 128, 128)
-        assert (t["BW"], t["BH"], t["MS"], t["NT"], t["SA"], t["SB"]) == (32, 4, 1, 64, 2, 3)
+        assert (t["MS"], t["NT"], t["SA"], t["SB"], t["mode"]) == (1, 64, 2, 3, 1)
     finally:
         qvae.qvae_set_conv_tiling()
     with pytest.raises(qvae.QvaeError):
-        qvae.qvae_set_conv_tiling(BW=24)
+        qvae.qvae_set_conv_tiling(MS=5)
     with pytest.raises(qvae.QvaeError):
         qvae.qvae_set_conv_tiling(NT=48)
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(MS=3, NT=256)
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(mode=3)

@@ -161,8 +161,11 @@ def conv_case(q, shape, seed, tiling=None, outliers=False, drift=False):
     return assert_bf16_close(dev_bits(out), ref["out"])
 
 
-TILINGS = [None, dict(BW=8), dict(BW=32), dict(BW=64), dict(BW=128), dict(MS=1),
-           dict(MS=1, BW=32, SA=1, SB=1), dict(NT=32), dict(SA=2, SB=3), dict(MS=2, BW=8, SA=1, SB=2)]
+TILINGS = [None,
+           dict(mode=1), dict(mode=1, MS=1), dict(mode=1, MS=3), dict(mode=1, MS=4, NT=64, SA=1, SB=2),
+           dict(mode=1, MS=1, SA=1, SB=1), dict(mode=1, NT=32),
+           dict(mode=2), dict(mode=2, MS=1), dict(mode=2, MS=2), dict(mode=2, MS=3), dict(mode=2, MS=4),
+           dict(mode=2, MS=1, SA=1, SB=1), dict(mode=2, NT=32), dict(mode=2, MS=2, NT=64, SA=2, SB=9)]
 
 
 @pytest.mark.parametrize("tiling", TILINGS)
@@ -180,14 +183,16 @@ def test_conv_tilings_exact(q, tiling):
     synth.LayerShape(160, 256, 8, 40),                # partial chunk of 32, NT = 256
     synth.LayerShape(96, 320, 6, 6),                  # NT = 160
 ])
-def test_conv_shapes_exact(q, shape):
-    conv_case(q, shape, seed=shape.Cin * 7 + shape.H)
+@pytest.mark.parametrize("mode", [1, 2])
+def test_conv_shapes_exact(q, shape, mode):
+    conv_case(q, shape, seed=shape.Cin * 7 + shape.H, tiling=dict(mode=mode))
 
 
 @pytest.mark.parametrize("H,W,T", [(1, 1, 1), (1, 2, 3), (2, 1, 2), (3, 5, 1), (5, 3, 2), (7, 9, 3),
                                    (9, 7, 1), (17, 17, 2), (1, 130, 1), (130, 1, 1)])
 def test_conv_tiny_and_odd(q, H, W, T):
-    conv_case(q, synth.LayerShape(32, 32, H, W, T=T), seed=H * 100 + W * 10 + T)
+    conv_case(q, synth.LayerShape(32, 32, H, W, T=T), seed=H * 100 + W * 10 + T, tiling=dict(mode=1))
+    conv_case(q, synth.LayerShape(32, 32, H, W, T=T), seed=H * 100 + W * 10 + T, tiling=dict(mode=2))
 
 
 def test_conv_outliers_and_drift(q):

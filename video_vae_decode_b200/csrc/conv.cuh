@@ -12,23 +12,37 @@
 // with zeros outside the tensor (two leading causal frames, one pixel of
 // spatial padding).  GEMM view: M = output pixels, N = Cout, K = taps x Cin.
 //
-// Tiling.  A CTA tile is MS sub-tiles of 128 pixels (BH rows x BW columns of
-// one frame, stacked vertically) by NT output channels.  For each real
-// temporal tap kt, each kw and each 128-channel chunk, one TMA box of
-// (MS*BH + 2) rows x BW pixels x 128 channels is loaded once (the tensor map's
-// out-of-bounds fill supplies the spatial zero padding); the three kh taps
-// are then the same box read at row offsets 0, 1, 2 -- a shift of BW*128
-// bytes, a whole number of 1024-byte swizzle atoms -- so the halo rows are
-// shared instead of reloaded.  Temporal taps that meet a causal zero frame are
-// skipped, not computed.  Weights come pre-packed in the MMA's swizzled K-major
-// layout and are streamed per (tap, chunk) with plain bulk copies.
+// Tiling.  A CTA tile is MS sub-tiles of 128 output pixels -- 16 image rows
+// x 8 columns of one frame, stacked vertically -- by NT output channels.  For
+// each real temporal tap kt and each 128-channel chunk, ONE TMA box of
+// (16*MS + 2) rows x 10 columns x 128 channels is loaded (the tensor map's
+// out-of-bounds fill supplies the zero padding).  In shared memory a pixel is
+// one 128-byte line of the tensor cores' 128-byte-swizzled K-major layout, and
+// an 8-pixel image row is one 8-line core-matrix group; with a group stride of
+// 10 lines (the box width) every one of the nine spatial taps (kh, kw) is the
+// same box read from line (kh * 10 + kw) on.  The swizzle is a function of the
+// absolute shared-memory address, so any line offset is a valid operand start:
+// the halo is loaded once and reused nine times.  Temporal taps that meet a
+// causal zero frame are skipped, not computed.  Weights come pre-packed in the
+// MMA's swizzled K-major layout and stream one tap at a time by 2-D TMA.
 //
-// Warp roles (192 threads): warp 0 issues the TMA / bulk copies, warp 1
-// issues tcgen05.mma (one thread) and owns the TMEM allocation, warps 2-5 run
-// the epilogue: tcgen05.ld of their 32 TMEM lanes, rescale + bias + bf16,
-// 16-byte stores.  Tiles are scheduled persistently (static stride); with
-// MS*NT <= 256 TMEM columns the accumulator is double-buffered so the
-// epilogue of one tile overlaps the main loop of the next.
+// CTA pairs.  With kPair the kernel runs as 2-CTA clusters on the tensor
+// cores' cta_group::2 path: one MMA covers M = 256 (128 pixels in each CTA)
+// by NT channels; each CTA loads its own activation box and HALF of every
+// weight tile (NT/2 rows), so weight traffic and shared-memory reads per
+// multiply-add halve.  Every load of both CTAs is counted on the leader CTA's
+// barriers; the leader issues the MMAs and its commits arrive on the barriers
+// of both CTAs; each CTA's epilogue drains its own TMEM rows.
+//
+// Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 issues tcgen05.mma
+// (one thread) and owns the TMEM allocation, warps 2-5 run the epilogue:
+// tcgen05.ld of their 32 TMEM lanes, rescale + bias + bf16, staged through
+// shared memory and written with TMA stores.  Tiles are scheduled
+// persistently (static stride); with MS*NT <= 256 TMEM columns the
+// accumulator is double-buffered so the epilogue of one tile overlaps the
+// main loop of the next.
+// Launched as a programmatic dependent of the activation quantiser: the
+// prologue and the first weight loads overlap its tail.
 #pragma once
 
 #include <cuda.h>
@@ -39,30 +53,40 @@
 
 namespace qvae {
 
+constexpr int kTileW = 8;       // output columns per tile = one 8-line core-matrix group
+constexpr int kTileRows = 16;   // image rows per 128-pixel sub-tile
+constexpr int kBoxW = kTileW + 2;
+constexpr uint32_t kGroupStride = kBoxW * 128u;  // bytes between image rows of the box
+
 struct ConvArgs {
   int N, T, H, W, Cin, Cout;
-  int BW, BH, MS, NT;         // tile geometry (BW * BH == 128)
-  int tiles_w, tiles_h, tiles_n, num_tiles;
+  int MS, NT;                 // sub-tiles per CTA tile, output channels per CTA tile
+  int tiles_w, tiles_h, tiles_n, num_tiles;  // tiles_h counts CTA-pair row bands in pair mode
   int nchunks, last_ksteps;   // 128-channel chunks; 32-channel k-steps in the last one
   int SA, SB, acc_stages;     // pipeline depths
-  uint32_t a_stage_bytes, b_stage_bytes, tmem_cols;
-  const int8_t* wq;           // packed weights
+  uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
+  uint32_t a_box_bytes;       // bytes one activation box delivers
+  uint32_t b_stage_bytes;     // weight rows this CTA loads per tap x 128 B
+  uint32_t tmem_cols;
   const float* x_scale;       // device scalar
   const float* w_scale;       // [Cout]
   const __nv_bfloat16* bias;  // [Cout] or null
-  __nv_bfloat16* out;         // [N,T,H,W,Cout]
   int32_t* acc_out;           // [N,T,H,W,Cout] (accumulator mode)
   uint64_t wait_limit_ns;
 };
 
 constexpr int kConvThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
+constexpr uint32_t kEpiStageBytes = 4096;  // per epilogue warp: 2 buffers x 32 pixels x 64 B
 
 struct TileCoord {
   int n, t, h0, w0, co0;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const ConvArgs& a, int tile) {
+// Tile -> coordinates.  In pair mode a tile is a band of 2*MS sub-tiles
+// shared by the two CTAs of a cluster; h0 is this CTA's first row.
+template <bool kPair>
+__device__ __forceinline__ TileCoord decode_tile(const ConvArgs& a, int tile, uint32_t rank) {
   TileCoord c;
   int r = tile;
   const int tn = r % a.tiles_n;
@@ -73,15 +97,17 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvArgs& a, int tile) {
   r /= a.tiles_h;
   c.t = r % a.T;
   c.n = r / a.T;
-  c.h0 = th * a.MS * a.BH;
-  c.w0 = tw * a.BW;
+  const int band = a.MS * kTileRows;
+  c.h0 = kPair ? (th * 2 + static_cast<int>(rank)) * band : th * band;
+  c.w0 = tw * kTileW;
   c.co0 = tn * a.NT;
   return c;
 }
 
-template <bool kAcc32>
+template <bool kAcc32, bool kPair>
 __global__ void __launch_bounds__(kConvThreads, 1)
-    conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const ConvArgs a) {
+    conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -89,7 +115,8 @@ __global__ void __launch_bounds__(kConvThreads, 1)
 
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
-  const uint32_t bars = b_ring + a.SB * a.b_stage_bytes;  // 8-byte mbarriers
+  const uint32_t epi_stage = b_ring + a.SB * a.b_stage_bytes;  // 1024-aligned
+  const uint32_t bars = epi_stage + 4 * kEpiStageBytes;        // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 16;
@@ -100,6 +127,10 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   float* const epi_smem = reinterpret_cast<float*>(misc + 16);  // 4 warps x 2 x NT floats
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;      // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int first_tile = kPair ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tile_step = kPair ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.SA; ++i) {
@@ -112,116 +143,182 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, 4);  // one arrive per epilogue warp
+      mbar_init(acc_empty + 8 * i, kPair ? 8 : 4);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), a.tmem_cols);
+  if (warp == 1) {
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), a.tmem_cols);
+    } else {
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), a.tmem_cols);
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) {
+    cluster_sync();  // both CTAs' barriers exist before either signals the other
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t limit = a.wait_limit_ns;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
+    // Weights do not depend on the preceding kernel: the first weight stages
+    // are filled before waiting for the activation codes.
     prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
     uint32_t as = 0, ap = 0, bs = 0, bp = 0;
     uint32_t a_armed = 0, a_par = 0, b_armed = 0, b_par = 0;  // per-stage bitmasks
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(a, tile);
+    const uint32_t tx_mult = kPair ? 2u : 1u;                 // bytes both CTAs deliver
+    int preissued = 0;
+    auto load_b = [&](const TileCoord& c, int kt, int ch, int tap9) -> bool {
+      if (!mbar_wait(b_empty + 8 * bs, bp ^ 1, abort_flag, limit, kErrTimeoutProducer)) return false;
+      const int tap = kt * 9 + tap9;  // (kt * 3 + kh) * 3 + kw
+      const int row = (tap * a.nchunks + ch) * a.Cout + c.co0 + static_cast<int>(rank) * (a.NT / 2);
+      const uint32_t bar = b_full + 8 * bs;
+      if (leader) mbar_arrive_expect_tx(bar, a.b_stage_bytes * tx_mult);
+      if (kPair) {
+        tma_load_2d_pair(b_ring + bs * a.b_stage_bytes, &tmap_w, map_to_cta(bar, 0), 0, row);
+      } else {
+        tma_load_2d(b_ring + bs * a.b_stage_bytes, &tmap_w, bar, 0, row);
+      }
+      b_armed |= 1u << bs;
+      b_par = (b_par & ~(1u << bs)) | (bp << bs);
+      if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
+      return true;
+    };
+    bool waited = false;
+    for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
+      const TileCoord c = decode_tile<kPair>(a, tile, rank);
       const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
-      for (int kt = kt_lo; kt < 3; ++kt)
-        for (int kw = 0; kw < 3; ++kw)
-          for (int ch = 0; ch < a.nchunks; ++ch) {
-            if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
-            mbar_arrive_expect_tx(a_full + 8 * as, a.a_stage_bytes);
-            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, a_full + 8 * as, ch * 128,
-                        c.w0 + kw - 1, c.h0 - 1, c.t + kt - 2, c.n);
-            a_armed |= 1u << as;
-            a_par = (a_par & ~(1u << as)) | (ap << as);
-            if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
-            for (int kh = 0; kh < 3; ++kh) {
-              if (!mbar_wait(b_empty + 8 * bs, bp ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
-              const int tap = (kt * 3 + kh) * 3 + kw;
-              const int8_t* src = a.wq + (static_cast<int64_t>(tap * a.nchunks + ch) * a.Cout + c.co0) * 128;
-              mbar_arrive_expect_tx(b_full + 8 * bs, a.b_stage_bytes);
-              bulk_load(b_ring + bs * a.b_stage_bytes, src, a.b_stage_bytes, b_full + 8 * bs);
-              b_armed |= 1u << bs;
-              b_par = (b_par & ~(1u << bs)) | (bp << bs);
-              if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
-            }
+      const int nkb = (3 - kt_lo) * a.nchunks;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int kt = kt_lo + kb / a.nchunks, ch = kb % a.nchunks;
+        if (!waited) {
+          for (; preissued < a.SB && preissued < 9; ++preissued)
+            if (!load_b(c, kt, ch, preissued)) goto producer_done;
+          grid_dependency_wait();
+          waited = true;
+        }
+        if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
+        {
+          const uint32_t bar = a_full + 8 * as;
+          if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
+          if (kPair) {
+            tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * 128, c.w0 - 1,
+                             c.h0 - 1, c.t + kt - 2, c.n);
+          } else {
+            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1,
+                        c.t + kt - 2, c.n);
           }
+        }
+        a_armed |= 1u << as;
+        a_par = (a_par & ~(1u << as)) | (ap << as);
+        if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
+        for (int i = preissued; i < 9; ++i)
+          if (!load_b(c, kt, ch, i)) goto producer_done;
+        preissued = 0;
+      }
     }
   producer_done:
-    if (*abort_flag) {
-      // Let every copy this thread started land before the CTA exits.
+    if (*abort_flag && leader) {
+      // Let every copy counted on this CTA's barriers land before it exits.
       int dummy = 0;
       for (int i = 0; i < a.SA; ++i)
         if (a_armed >> i & 1) mbar_wait(a_full + 8 * i, a_par >> i & 1, &dummy, limit, kErrTimeoutDrain);
       for (int i = 0; i < a.SB; ++i)
         if (b_armed >> i & 1) mbar_wait(b_full + 8 * i, b_par >> i & 1, &dummy, limit, kErrTimeoutDrain);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_i8(128, a.NT);
-    const uint32_t row_shift = static_cast<uint32_t>(a.BW) * 128u;  // one image row of the box
+    const uint32_t idesc = idesc_i8(kPair ? 256 : 128, a.NT);
     uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
     bool issued = false;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(a, tile);
+    auto commit = [&](uint32_t bar) {
+      if (kPair) {
+        mma_commit_pair_multicast(bar, 0x3);
+      } else {
+        mma_commit(bar);
+      }
+    };
+    for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
+      const TileCoord c = decode_tile<kPair>(a, tile, rank);
       const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
+      const int nkb = (3 - kt_lo) * a.nchunks;
       if (!mbar_wait(acc_empty + 8 * cs, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
       tc_fence_after();
       const uint32_t d_tile = tmem_base + cs * static_cast<uint32_t>(a.MS * a.NT);
       bool first = true;
-      for (int kt = kt_lo; kt < 3; ++kt)
-        for (int kw = 0; kw < 3; ++kw)
-          for (int ch = 0; ch < a.nchunks; ++ch) {
-            if (!mbar_wait(a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
-            tc_fence_after();
-            const int ksteps = (ch == a.nchunks - 1) ? a.last_ksteps : 4;
-            const uint32_t a_stage = a_ring + as * a.a_stage_bytes;
-            for (int kh = 0; kh < 3; ++kh) {
-              if (!mbar_wait(b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
-              tc_fence_after();
-              const uint32_t b_stage = b_ring + bs * a.b_stage_bytes;
-              for (int s = 0; s < a.MS; ++s) {
-                const uint32_t a_rows = a_stage + static_cast<uint32_t>(s * a.BH + kh) * row_shift;
-                for (int k = 0; k < ksteps; ++k) {
-                  mma_i8(d_tile + static_cast<uint32_t>(s * a.NT), sw128_kmajor_desc(a_rows + 32u * k),
-                         sw128_kmajor_desc(b_stage + 32u * k), idesc, (first && k == 0) ? 0u : 1u);
-                  issued = true;
-                }
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int ch = kb % a.nchunks;
+        if (!mbar_wait(a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
+        tc_fence_after();
+        const int ksteps = (ch == a.nchunks - 1) ? a.last_ksteps : 4;
+        const uint32_t a_stage = a_ring + as * a.a_stage_bytes;
+        for (int tap9 = 0; tap9 < 9; ++tap9) {
+          const int kh = tap9 / 3, kw = tap9 % 3;
+          if (!mbar_wait(b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
+          tc_fence_after();
+          const uint32_t b_stage = b_ring + bs * a.b_stage_bytes;
+          for (int s = 0; s < a.MS; ++s) {
+            // sub-tile s, tap (kh, kw): box row s*16 + kh, column kw
+            const uint32_t a_rows = a_stage + static_cast<uint32_t>(s * kTileRows + kh) * kGroupStride +
+                                    static_cast<uint32_t>(kw) * 128u;
+            for (int k = 0; k < ksteps; ++k) {
+              const uint64_t ad = sw128_kmajor_desc(a_rows + 32u * k, kGroupStride);
+              const uint64_t bd = sw128_kmajor_desc(b_stage + 32u * k, 1024u);
+              const uint32_t acc = (first && k == 0) ? 0u : 1u;
+              if (kPair) {
+                mma_i8_pair(d_tile + static_cast<uint32_t>(s * a.NT), ad, bd, idesc, acc);
+              } else {
+                mma_i8(d_tile + static_cast<uint32_t>(s * a.NT), ad, bd, idesc, acc);
               }
-              first = false;
-              mma_commit(b_empty + 8 * bs);
-              if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
+              issued = true;
             }
-            mma_commit(a_empty + 8 * as);
-            if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
           }
-      mma_commit(acc_full + 8 * cs);
+          first = false;
+          commit(b_empty + 8 * bs);
+          if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
+        }
+        commit(a_empty + 8 * as);
+        if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
+      }
+      commit(acc_full + 8 * cs);
       if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
     }
   mma_done:
     if (*abort_flag && issued) {
       // Wait for the tensor cores to finish what was issued before TMEM is freed.
       int dummy = 0;
-      mma_commit(drain_bar);
+      if (kPair) {
+        mma_commit_pair(drain_bar);
+      } else {
+        mma_commit(drain_bar);
+      }
       mbar_wait(drain_bar, 0, &dummy, limit, kErrTimeoutDrain);
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;          // tile row = TMEM lane
+    // Warp q owns TMEM lanes 32q..32q+31 = tile rows 4q..4q+3 x 8 columns.  Each
+    // 32-channel slice is converted, staged in shared memory (64-byte swizzle)
+    // and written by one TMA store of a 32 x 8 x 4 box, which also drops the
+    // rows and columns beyond the image edge.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
     float* const sc = epi_smem + (warp - 2) * 2 * a.NT;
     float* const bi = sc + a.NT;
+    const uint32_t stage = epi_stage + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;
+    const uint32_t empty_leader = kPair ? map_to_cta(acc_empty, 0) : acc_empty;
+    uint32_t buf = 0;
     uint32_t cs = 0, cp = 0;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(a, tile);
+    grid_dependency_wait();
+    for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
+      const TileCoord c = decode_tile<kPair>(a, tile, rank);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(acc_full + 8 * cs, cp, abort_flag, limit, kErrTimeoutEpilogue);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -237,16 +334,15 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cs * static_cast<uint32_t>(a.MS * a.NT);
       for (int s = 0; s < a.MS; ++s) {
-        const int h = c.h0 + s * a.BH + row / a.BW;
-        const int w = c.w0 + row % a.BW;
-        const bool valid = h < a.H && w < a.W;
-        const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
+        const int h = c.h0 + s * kTileRows + row / kTileW;
+        const int w = c.w0 + row % kTileW;
         for (int cc = 0; cc < a.NT; cc += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(s * a.NT + cc), v);
           tmem_ld_wait();
-          if (!valid) continue;
           if (kAcc32) {
+            if (h >= a.H || w >= a.W) continue;
+            const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
             int4* dst = reinterpret_cast<int4*>(a.acc_out + pix * a.Cout + c.co0 + cc);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -263,26 +359,59 @@ __global__ void __launch_bounds__(kConvThreads, 1)
               const __nv_bfloat162 p = __floats2bfloat162_rn(y0, y1);
               packed[e] = *reinterpret_cast<const uint32_t*>(&p);
             }
-            uint4* dst = reinterpret_cast<uint4*>(a.out + pix * a.Cout + c.co0 + cc);
+            // the store issued two slices ago read this buffer: let it finish
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            const uint32_t line = stage + buf * 2048u + static_cast<uint32_t>(lane) * 64u;
+            const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+            for (int k = 0; k < 4; ++k)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((k ^ swz) << 4)),
+                           "r"(packed[4 * k]), "r"(packed[4 * k + 1]), "r"(packed[4 * k + 2]),
+                           "r"(packed[4 * k + 3])
+                           : "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_5d(&tmap_out, stage + buf * 2048u, c.co0 + cc, c.w0,
+                           c.h0 + s * kTileRows + q * 4, c.t, c.n);
+              bulk_commit_group();
+            }
+            buf ^= 1u;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + 8 * cs);
+      if (lane == 0) {
+        if (kPair) {
+          mbar_arrive_cluster(empty_leader + 8 * cs);
+        } else {
+          mbar_arrive(acc_empty + 8 * cs);
+        }
+      }
       if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
     }
+    if (!kAcc32 && lane == 0) bulk_wait_group<0>();
   }
 
+  // Reconverge every warp (one lane of warps 0 and 1 ran a role alone) before
+  // the warp-aligned block / cluster barrier.
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (kPair) {
+    cluster_sync();  // neither CTA leaves while its partner may still touch its memory
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, a.tmem_cols);
+    if (kPair) {
+      tmem_dealloc_pair(tmem_base, a.tmem_cols);
+    } else {
+      tmem_dealloc(tmem_base, a.tmem_cols);
+    }
   }
 }
 

@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace qvae {
 
 // |bf16| ordering equals the unsigned ordering of its low 15 bits (finite
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __
                                                                   int64_t numel,
                                                                   uint32_t* __restrict__ partial) {
   __shared__ uint32_t red[kActThreads / 32];
+  grid_dependents_launch();  // the quantiser may start its prologue
   uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
   int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
@@ -129,6 +132,8 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
     const uint32_t* __restrict__ partial, int npartial, uint4* __restrict__ xq,
     int8_t* __restrict__ xq_bytes, float* __restrict__ x_scale) {
   __shared__ uint32_t red[kActThreads / 32];
+  grid_dependents_launch();  // the convolution may start its prologue
+  grid_dependency_wait();    // the partial maxima of the previous kernel are complete
   uint32_t m = 0;
   for (int k = threadIdx.x; k < npartial; k += kActThreads) m = max(m, partial[k]);
   m = block_max_u32<kActThreads>(m, red);

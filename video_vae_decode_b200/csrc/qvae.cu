@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/qvae.h"
 #include "conv.cuh"
@@ -24,11 +25,12 @@ using qvae::ConvArgs;
 
 thread_local std::string t_last_error;
 uint64_t g_wait_limit_ns = 2000000000ull;
-int32_t g_force[5] = {0, 0, 0, 0, 0};  // BW, MS, NT, SA, SB
+int32_t g_force[5] = {0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair)
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
-bool g_conv_attr_set[kMaxDevices][2] = {};
+bool g_conv_attr_set[kMaxDevices][4] = {};
+int g_max_clusters[kMaxDevices] = {0};
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
 
@@ -79,80 +81,106 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // ------------------------------------------------------------------ tiling
 
 struct Tiling {
-  int BW, BH, MS, NT, SA, SB, acc_stages;
-  uint32_t a_stage_bytes, b_stage_bytes, tmem_cols, smem_bytes;
-  int tiles_w, tiles_h, tiles_n, num_tiles;
+  bool pair;
+  int MS, NT, SA, SB, acc_stages;
+  uint32_t a_stage_bytes, a_box_bytes, b_stage_bytes, tmem_cols, smem_bytes;
+  int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
+  double est_cycles;
 };
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 uint32_t smem_needed(const Tiling& t) {
   const uint32_t bars = 8 * qvae::kMaxStages * 4 + 16 + 16 + 8;
-  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + bars + 16 + 4 * 2 * t.NT * 4;
+  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + 4 * qvae::kEpiStageBytes + bars + 16 +
+         4 * 2 * t.NT * 4;
 }
 
-int choose_nt(int Cout, int forced) {
-  if (forced) return (forced % 32 == 0 && forced <= 256 && Cout % forced == 0) ? forced : 0;
-  for (int n = static_cast<int>(ceil_div(Cout, 256)); n <= Cout / 32; ++n)
-    if (Cout % n == 0 && (Cout / n) % 32 == 0) return Cout / n;
-  return 0;
-}
-
-int make_tiling(const qvae_shape& s, Tiling* t) {
-  t->NT = choose_nt(s.Cout, g_force[2]);
-  if (t->NT == 0) return QVAE_ERR_SHAPE;
-  t->MS = g_force[1] ? g_force[1] : 2;
-  if (t->MS != 1 && t->MS != 2) return QVAE_ERR_ARG;
-  // Tile width: least padded area, then the narrower tile (less halo per box).
-  static const int kWidths[5] = {16, 32, 8, 64, 128};
-  int best_bw = 0;
-  int64_t best_area = 0;
-  for (int bw : kWidths) {
-    if (g_force[0] && bw != g_force[0]) continue;
-    const int rows = t->MS * (128 / bw);
-    const int64_t area = ceil_div(s.W, bw) * bw * ceil_div(s.H, rows) * rows;
-    if (best_bw == 0 || area < best_area) { best_bw = bw; best_area = area; }
+// Pipeline depths for a geometry: the deepest weight ring (up to 9 stages,
+// one tap each) next to two activation stages, else the best that fits.
+bool fit_stages(Tiling* t) {
+  if (g_force[2] || g_force[3]) {
+    t->SA = g_force[2] ? g_force[2] : 2;
+    t->SB = g_force[3] ? g_force[3] : 4;
+    return smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit);
   }
-  if (best_bw == 0) return QVAE_ERR_ARG;
-  t->BW = best_bw;
-  t->BH = 128 / best_bw;
-  t->a_stage_bytes = static_cast<uint32_t>(t->MS * t->BH + 2) * t->BW * 128u;
-  t->b_stage_bytes = static_cast<uint32_t>(t->NT) * 128u;
-  const int acc_cols = t->MS * t->NT;
+  for (int sa = 2; sa >= 1; --sa) {
+    t->SA = sa;
+    for (t->SB = 9; t->SB >= 2; --t->SB)
+      if (smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit)) return true;
+  }
+  return false;
+}
+
+// Relative cost of a geometry on `sms` SMs, in SM cycles: waves x the time of
+// a CTA tile.  A tile is its weight stages (one per tap and 128-channel chunk),
+// each MS x k-steps MMAs of 128 x NT x 32 at the measured cycles per MMA for
+// that N plus a measured ~330-cycle handshake, and the epilogue when the
+// accumulator cannot be double-buffered.  A CTA pair shares weight loads but
+// measured no faster than single CTAs here, so it is charged slightly more.
+double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
+  double taps_t = 0;
+  for (int64_t f = 0; f < std::min<int64_t>(s.T, 2); ++f) taps_t += static_cast<double>(f + 1);
+  if (s.T > 2) taps_t += 3.0 * (s.T - 2);
+  taps_t /= s.T;
+  // cycles per MMA measured with random data: N=96 86, 128 91, 192 109, 256 143
+  const double mma = std::max(0.52 * t.NT + 8.0, 60.0 + 0.17 * t.NT);
+  const int nchunks = (s.Cin + 127) / 128;
+  const double ksteps_total = s.Cin / 32.0;
+  const double stages = taps_t * 9.0 * nchunks;
+  const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 330.0 + 1500.0 +
+                          (t.acc_stages == 1 ? 6.0 * t.MS * t.NT : 0.0);
+  const double slots = t.pair ? std::floor(sms / 2.0) : sms;
+  const double waves = std::ceil(static_cast<double>(t.num_tiles) / slots);
+  return (waves * per_tile + (t.acc_stages == 1 ? 0.0 : 6.0 * t.MS * t.NT)) * (t.pair ? 1.05 : 1.0);
+}
+
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, Tiling* t) {
+  t->pair = pair;
+  t->MS = MS;
+  t->NT = NT;
+  t->ctas_per_tile = pair ? 2 : 1;
+  const int rows = MS * qvae::kTileRows + 2;
+  t->a_box_bytes = static_cast<uint32_t>(rows) * qvae::kGroupStride;
+  t->a_stage_bytes = (t->a_box_bytes + 1023u) & ~1023u;
+  t->b_stage_bytes = static_cast<uint32_t>(pair ? NT / 2 : NT) * 128u;
+  const int acc_cols = MS * NT;
+  if (acc_cols > 512) return QVAE_ERR_ARG;
   t->acc_stages = (2 * acc_cols <= 512) ? 2 : 1;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(t->acc_stages * acc_cols)) cols <<= 1;
   t->tmem_cols = cols;
-  if (g_force[3] || g_force[4]) {
-    t->SA = g_force[3] ? g_force[3] : 2;
-    t->SB = g_force[4] ? g_force[4] : 4;
-    if (t->SA < 1 || t->SA > qvae::kMaxStages || t->SB < 1 || t->SB > qvae::kMaxStages) return QVAE_ERR_ARG;
-  } else {
-    // Deepest pipeline that fits, about three weight stages per activation stage.
-    Tiling best = *t;
-    best.SA = 0;
-    for (int sa = 4; sa >= 2 && best.SA == 0; --sa) {
-      Tiling u = *t;
-      u.SA = sa;
-      for (u.SB = 8; u.SB >= 3 && smem_needed(u) > kSmemLimit; --u.SB) {}
-      if (smem_needed(u) <= kSmemLimit && u.SB >= std::min(8, 3 * sa - 1)) best = u;
-    }
-    if (best.SA == 0) {
-      best = *t;
-      best.SA = 2;
-      for (best.SB = 8; best.SB > 2 && smem_needed(best) > kSmemLimit; --best.SB) {}
-    }
-    *t = best;
-  }
+  if (!fit_stages(t)) return QVAE_ERR_UNSUPPORTED;
   t->smem_bytes = smem_needed(*t);
-  if (t->smem_bytes > kSmemLimit) return QVAE_ERR_UNSUPPORTED;
-  t->tiles_w = static_cast<int>(ceil_div(s.W, t->BW));
-  t->tiles_h = static_cast<int>(ceil_div(s.H, t->MS * t->BH));
-  t->tiles_n = s.Cout / t->NT;
+  t->tiles_w = static_cast<int>(ceil_div(s.W, qvae::kTileW));
+  t->tiles_h = static_cast<int>(ceil_div(s.H, MS * qvae::kTileRows * t->ctas_per_tile));
+  t->tiles_n = s.Cout / NT;
   const int64_t tiles = s.N * s.T * t->tiles_h * static_cast<int64_t>(t->tiles_w) * t->tiles_n;
-  if (tiles > INT32_MAX) return QVAE_ERR_SHAPE;
+  if (tiles > INT32_MAX / 2) return QVAE_ERR_SHAPE;
   t->num_tiles = static_cast<int>(tiles);
   return QVAE_OK;
+}
+
+int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148) {
+  bool found = false;
+  for (int mode = 1; mode <= 2; ++mode) {
+    if (g_force[4] && mode != g_force[4]) continue;
+    for (int ms = 1; ms <= 4; ++ms) {
+      if (g_force[0] && ms != g_force[0]) continue;
+      for (int nt = 32; nt <= std::min(256, s.Cout); nt += 32) {
+        if (s.Cout % nt) continue;
+        if (g_force[1] && nt != g_force[1]) continue;
+        Tiling u;
+        if (make_geometry(s, mode == 2, ms, nt, &u) != QVAE_OK) continue;
+        u.est_cycles = estimate_cycles(s, u, sms);
+        if (!found || u.est_cycles < t->est_cycles) {
+          *t = u;
+          found = true;
+        }
+      }
+    }
+  }
+  return found ? QVAE_OK : QVAE_ERR_UNSUPPORTED;
 }
 
 int check_shape(const qvae_shape* s) {
@@ -170,6 +198,53 @@ int check_shape(const qvae_shape* s) {
 
 int64_t pixels(const qvae_shape& s) { return s.N * s.T * s.H * s.W; }
 
+int encode_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, const cuuint64_t* dims,
+               const cuuint64_t* strides, const cuuint32_t* box, int rank, CUtensorMapSwizzle swizzle) {
+  auto encode = tensor_map_encoder();
+  if (!encode) {
+    t_last_error = "cuTensorMapEncodeTiled is not available from the driver";
+    return QVAE_ERR_CUDA;
+  }
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult cr = encode(map, dtype, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    char buf[128];
+    std::snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(cr));
+    t_last_error = buf;
+    return QVAE_ERR_CUDA;
+  }
+  return QVAE_OK;
+}
+
+// Launch as a programmatic dependent of the previous kernel on the stream:
+// the grid may start while its predecessor finishes and synchronises with
+// griddepcontrol.wait before touching the predecessor's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                             cudaStream_t stream, int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                 const int8_t* wq, const float* w_scale, const void* bias, void* out, int32_t* acc,
                 cudaStream_t stream) {
@@ -181,41 +256,56 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   if (!xq || !wq || (!acc_mode && (!x_scale || !w_scale || !out))) return QVAE_ERR_ARG;
   if (!aligned16(xq) || !aligned16(wq) || (out && !aligned16(out)) || (acc && !aligned16(acc)))
     return QVAE_ERR_ALIGN;
-  Tiling t;
-  rc = make_tiling(s, &t);
-  if (rc) return rc;
   int dev;
   rc = current_device(&dev);
   if (rc) return rc;
   int sms;
   rc = sm_count(dev, &sms);
   if (rc) return rc;
+  Tiling t;
+  rc = make_tiling(s, &t, sms);
+  if (rc) return rc;
 
-  auto encode = tensor_map_encoder();
-  if (!encode) {
-    t_last_error = "cuTensorMapEncodeTiled is not available from the driver";
-    return QVAE_ERR_CUDA;
+  CUtensorMap tmap_x, tmap_w, tmap_out;
+  {
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W),
+                                static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.T),
+                                static_cast<cuuint64_t>(s.N)};
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin),
+                                   static_cast<cuuint64_t>(s.W) * s.Cin,
+                                   static_cast<cuuint64_t>(s.H) * s.W * s.Cin,
+                                   static_cast<cuuint64_t>(s.T) * s.H * s.W * s.Cin};
+    const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(qvae::kBoxW),
+                               static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
+    rc = encode_map(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims, strides, box, 5,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
   }
-  CUtensorMap tmap;
-  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W),
-                              static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.T),
-                              static_cast<cuuint64_t>(s.N)};
-  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin),
-                                 static_cast<cuuint64_t>(s.W) * s.Cin,
-                                 static_cast<cuuint64_t>(s.H) * s.W * s.Cin,
-                                 static_cast<cuuint64_t>(s.T) * s.H * s.W * s.Cin};
-  const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(t.BW),
-                             static_cast<cuuint32_t>(t.MS * t.BH + 2), 1u, 1u};
-  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
-  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<int8_t*>(xq), dims,
-                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) {
-    char buf[128];
-    std::snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(cr));
-    t_last_error = buf;
-    return QVAE_ERR_CUDA;
+  {
+    // packed weights as rows of 128 bytes: [tap][chunk][Cout] rows
+    const int nchunks = (s.Cin + 127) / 128;
+    const cuuint64_t dims[2] = {128u, static_cast<cuuint64_t>(27) * nchunks * s.Cout};
+    const cuuint64_t strides[1] = {128u};
+    const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(t.pair ? t.NT / 2 : t.NT)};
+    rc = encode_map(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, dims, strides, box, 2,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+  }
+  if (!acc_mode) {
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cout), static_cast<cuuint64_t>(s.W),
+                                static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.T),
+                                static_cast<cuuint64_t>(s.N)};
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cout) * 2,
+                                   static_cast<cuuint64_t>(s.W) * s.Cout * 2,
+                                   static_cast<cuuint64_t>(s.H) * s.W * s.Cout * 2,
+                                   static_cast<cuuint64_t>(s.T) * s.H * s.W * s.Cout * 2};
+    // one epilogue warp's slice: 32 channels x 8 columns x 4 rows
+    const cuuint32_t box[5] = {32u, static_cast<cuuint32_t>(qvae::kTileW), 4u, 1u, 1u};
+    rc = encode_map(&tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, dims, strides, box, 5,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
+    if (rc) return rc;
+  } else {
+    tmap_out = tmap_x;  // unused by the accumulator variant
   }
 
   ConvArgs a;
@@ -225,8 +315,6 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.W = static_cast<int>(s.W);
   a.Cin = s.Cin;
   a.Cout = s.Cout;
-  a.BW = t.BW;
-  a.BH = t.BH;
   a.MS = t.MS;
   a.NT = t.NT;
   a.tiles_w = t.tiles_w;
@@ -239,33 +327,48 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.SB = t.SB;
   a.acc_stages = t.acc_stages;
   a.a_stage_bytes = t.a_stage_bytes;
+  a.a_box_bytes = t.a_box_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
-  a.wq = wq;
   a.x_scale = x_scale;
   a.w_scale = w_scale;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
-  a.out = static_cast<__nv_bfloat16*>(out);
   a.acc_out = acc;
   a.wait_limit_ns = g_wait_limit_ns;
 
-  const int grid = std::min(t.num_tiles, sms);
-  if (acc_mode) {
-    if (!g_conv_attr_set[dev][1]) {
-      QVAE_CUDA(cudaFuncSetAttribute(qvae::conv3d_w8a8_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-      g_conv_attr_set[dev][1] = true;
-    }
-    qvae::conv3d_w8a8_kernel<true><<<grid, qvae::kConvThreads, t.smem_bytes, stream>>>(tmap, a);
-  } else {
-    if (!g_conv_attr_set[dev][0]) {
-      QVAE_CUDA(cudaFuncSetAttribute(qvae::conv3d_w8a8_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-      g_conv_attr_set[dev][0] = true;
-    }
-    qvae::conv3d_w8a8_kernel<false><<<grid, qvae::kConvThreads, t.smem_bytes, stream>>>(tmap, a);
+  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0);
+  using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, qvae::ConvArgs);
+  const Kernel kernels[4] = {qvae::conv3d_w8a8_kernel<false, false>, qvae::conv3d_w8a8_kernel<true, false>,
+                             qvae::conv3d_w8a8_kernel<false, true>, qvae::conv3d_w8a8_kernel<true, true>};
+  const Kernel kernel = kernels[kidx];
+  if (!g_conv_attr_set[dev][kidx]) {
+    QVAE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    g_conv_attr_set[dev][kidx] = true;
   }
-  QVAE_CUDA(cudaGetLastError());
+  int grid;
+  if (t.pair) {
+    if (g_max_clusters[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * sms);
+      cfg.blockDim = dim3(qvae::kConvThreads);
+      cfg.dynamicSmemBytes = kSmemLimit;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      QVAE_CUDA(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg));
+      g_max_clusters[dev] = std::max(n, 1);
+    }
+    grid = 2 * std::min(t.num_tiles, g_max_clusters[dev]);
+  } else {
+    grid = std::min(t.num_tiles, sms);
+  }
+  QVAE_CUDA(launch_dependent(kernel, grid, qvae::kConvThreads, t.smem_bytes, stream, t.pair ? 2 : 1, tmap_x,
+                             tmap_w, tmap_out, a));
   return QVAE_OK;
 }
 
@@ -301,10 +404,10 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   const int64_t nvec2 = numel / 16;
   const int g2 = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>(ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * 2), 4LL * sms)));
-  qvae::act_quant_kernel<<<g2, qvae::kActThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), nvec2, static_cast<const uint16_t*>(x), numel, partial, g1,
-      reinterpret_cast<uint4*>(xq), xq, x_scale);
-  QVAE_CUDA(cudaGetLastError());
+  QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, stream, 1,
+                             static_cast<const uint4*>(x), nvec2, static_cast<const uint16_t*>(x), numel,
+                             static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
+                             x_scale));
   return QVAE_OK;
 }
 
@@ -397,7 +500,7 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
     int rc = check_shape(&L.shape);
     if (rc) return rc;
     Tiling t;
-    if ((rc = make_tiling(L.shape, &t))) return rc;
+    if ((rc = make_tiling(L.shape, &t))) return rc;  // the shape has a valid tiling
     if (!L.x || !L.out || !L.wq_packed || !L.w_scale) return QVAE_ERR_ARG;
     if (!aligned16(L.x) || !aligned16(L.out) || !aligned16(L.wq_packed)) return QVAE_ERR_ALIGN;
   }
@@ -450,16 +553,17 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return QVAE_OK;
 }
 
-int qvae_set_conv_tiling(int32_t BW, int32_t MS, int32_t NT, int32_t SA, int32_t SB) {
-  if (BW && BW != 8 && BW != 16 && BW != 32 && BW != 64 && BW != 128) return QVAE_ERR_ARG;
-  if (MS && MS != 1 && MS != 2) return QVAE_ERR_ARG;
+int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode) {
+  if (MS < 0 || MS > 4) return QVAE_ERR_ARG;
   if (NT && (NT % 32 || NT > 256 || NT < 32)) return QVAE_ERR_ARG;
+  if (MS && NT && MS * NT > 512) return QVAE_ERR_ARG;
   if (SA < 0 || SA > qvae::kMaxStages || SB < 0 || SB > qvae::kMaxStages) return QVAE_ERR_ARG;
-  g_force[0] = BW;
-  g_force[1] = MS;
-  g_force[2] = NT;
-  g_force[3] = SA;
-  g_force[4] = SB;
+  if (mode < 0 || mode > 2) return QVAE_ERR_ARG;
+  g_force[0] = MS;
+  g_force[1] = NT;
+  g_force[2] = SA;
+  g_force[3] = SB;
+  g_force[4] = mode;
   return QVAE_OK;
 }
 
@@ -467,15 +571,18 @@ int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7) {
   if (!out7) return QVAE_ERR_ARG;
   int rc = check_shape(shape);
   if (rc) return rc;
+  int sms = 148, dev;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) sm_count(dev, &sms);
+  cudaGetLastError();
   Tiling t;
-  if ((rc = make_tiling(*shape, &t))) return rc;
-  out7[0] = t.BW;
-  out7[1] = t.BH;
-  out7[2] = t.MS;
-  out7[3] = t.NT;
-  out7[4] = t.SA;
-  out7[5] = t.SB;
-  out7[6] = t.num_tiles;
+  if ((rc = make_tiling(*shape, &t, sms))) return rc;
+  out7[0] = t.MS;
+  out7[1] = t.NT;
+  out7[2] = t.SA;
+  out7[3] = t.SB;
+  out7[4] = t.acc_stages;
+  out7[5] = t.num_tiles * t.ctas_per_tile;
+  out7[6] = t.pair ? 2 : 1;
   return QVAE_OK;
 }
 

@@ -234,12 +234,12 @@ def qvae_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("qvae_selftest_wait_timeout", lib().qvae_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
-def qvae_set_conv_tiling(BW=0, MS=0, NT=0, SA=0, SB=0) -> None:
-    _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(BW, MS, NT, SA, SB))
+def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0) -> None:
+    _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(MS, NT, SA, SB, mode))
 
 
 def qvae_get_conv_tiling(N, T, H, W, Cin, Cout) -> dict:
     shp = make_shape(N, T, H, W, Cin, Cout)
     out = (ctypes.c_int32 * 7)()
     _check("qvae_get_conv_tiling", lib().qvae_get_conv_tiling(ctypes.byref(shp), out))
-    return dict(zip(("BW", "BH", "MS", "NT", "SA", "SB", "tiles"), list(out)))
+    return dict(zip(("MS", "NT", "SA", "SB", "acc_buffers", "ctas", "mode"), list(out)))
