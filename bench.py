@@ -46,6 +46,21 @@ def parse():
     return ap.parse_args()
 
 
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own independently seeded layer (weak scaling)."""
+    return base_seed + rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (a no-op on one process)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -232,7 +247,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
 
     wl = synth.WORKLOADS[args.workload]
-    layer = synth.draw_workload(args.workload, seed=wl.seed + rank, only=[args.layer])[0]
+    layer = synth.draw_workload(args.workload, seed=rank_seed(wl.seed, rank), only=[args.layer])[0]
     s = layer.shape
     w, b = layer.w.to(dev), layer.bias.to(dev)
     packed0, s_w = qvae.quantize_weights(w)                # once, as at model load
@@ -320,10 +335,7 @@ def run_ours(args):
     e2e_ms = e2e_a.elapsed_time(e2e_b) / e2e_steps
 
     ops = s.ops()
-    t = torch.tensor([total_ms, e2e_ms, statistics.mean(conv_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max, e2e_ms_max, conv_ms_max = t.tolist()
+    total_ms_max, e2e_ms_max, conv_ms_max = max_over_ranks([total_ms, e2e_ms, statistics.mean(conv_ms)], dev)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
