@@ -106,6 +106,28 @@ size_t qvae_act_workspace_bytes(int64_t numel);
 int qvae_act_absmax_quant(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * qvae_act_absmax_quant without a workspace argument: the same quantisation
+ * and outputs, with its scratch (the partial maxima) in a fixed 16 KiB device
+ * array inside this library instead of caller memory.  The release note has
+ * no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory -- a host runtime that owns every device buffer and
+ * hands a layer only its input and output tensors, or a decode loop that may
+ * not call cudaMalloc mid-stream (it can block, synchronise the device or fail
+ * under memory pressure).  It allocates nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - The array holds 4096 partial maxima; a launch needing more (a GPU with
+ *     more than 1024 SMs) returns QVAE_ERR_UNSUPPORTED with a message.
+ *   - Every call on a device shares the one array and leaves the last call's
+ *     partial maxima in it; nothing needs clearing because every slot a call
+ *     reads is written earlier in the same call.  Calls that overlap on the
+ *     GPU (different streams, different host threads) race on the array.
+ */
+int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
+                                  void* stream);
+
 /* ---------------------------------------------------------- convolution -- */
 
 /*

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <mutex>
 #include <string>
 #include <utility>
 
@@ -415,6 +416,36 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
+// ====================================================== fixed device scratch
+// For callers that cannot allocate device memory, qvae_act_absmax_quant_noalloc
+// keeps the activation quantiser's partial maxima in this fixed array instead
+// of a caller workspace.  Every GPU that loads the library holds it (16 KiB)
+// until the process exits.
+namespace {
+
+constexpr int kStaticPartialSlots = 4096;  // one 32-bit partial maximum per absmax CTA
+static __device__ __align__(256) uint32_t g_static_partials[kStaticPartialSlots];
+
+void* g_static_partials_addr[kMaxDevices] = {};
+std::mutex g_static_mutex;
+
+// The device address of the array on the current device.  In host code the
+// array's name is only a host-side handle, so the address is looked up once per
+// device (with that device current) and cached.
+int static_partials(int dev, uint32_t** out) {
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_partials_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_partials);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static partial maxima)");
+    g_static_partials_addr[dev] = p;
+  }
+  *out = static_cast<uint32_t*>(g_static_partials_addr[dev]);
+  return QVAE_OK;
+}
+
+}  // namespace
+
 // ================================================================== C ABI
 
 extern "C" {
@@ -480,6 +511,45 @@ int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
   if (!acc) return QVAE_ERR_ARG;
   return launch_conv(shape, xq, nullptr, wq_packed, nullptr, nullptr, nullptr, acc,
                      static_cast<cudaStream_t>(stream));
+}
+
+int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
+                                  void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (numel < 0 || !x_scale) return QVAE_ERR_ARG;
+  if (numel == 0) {
+    QVAE_CUDA(cudaMemsetAsync(x_scale, 0, sizeof(float), st));
+    return QVAE_OK;
+  }
+  if (!x_bf16 || !xq) return QVAE_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(xq)) return QVAE_ERR_ALIGN;
+  int dev, sms, rc;
+  if ((rc = current_device(&dev))) return rc;
+  if ((rc = sm_count(dev, &sms))) return rc;
+  const int g1 = act_grid(numel, sms);
+  if (g1 > kStaticPartialSlots) {
+    char buf[160];
+    std::snprintf(buf, sizeof buf,
+                  "this launch needs %d partial-maximum slots; the fixed scratch holds %d", g1,
+                  kStaticPartialSlots);
+    t_last_error = buf;
+    return QVAE_ERR_UNSUPPORTED;
+  }
+  uint32_t* partial = nullptr;
+  if ((rc = static_partials(dev, &partial))) return rc;
+  // Same two kernels as qvae_act_absmax_quant; every slot the second reads is
+  // written by the first in this call, so nothing needs clearing.
+  qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, st>>>(
+      static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, partial);
+  QVAE_CUDA(cudaGetLastError());
+  const int64_t nvec2 = numel / 16;
+  const int g2 = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * 2), 4LL * sms)));
+  QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, st, 1,
+                             static_cast<const uint4*>(x_bf16), nvec2, static_cast<const uint16_t*>(x_bf16),
+                             numel, static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
+                             x_scale));
+  return QVAE_OK;
 }
 
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {

@@ -27,6 +27,7 @@ EXPORTS = (
     "qvae_causal_conv3d_w8a8", "qvae_causal_conv3d_w8a8_acc32", "qvae_decode_workspace_bytes",
     "qvae_decode_layers", "qvae_get_error", "qvae_set_wait_limit_ns",
     "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling",
+    "qvae_act_absmax_quant_noalloc",
 )
 
 
@@ -66,6 +67,7 @@ def lib():
             "qvae_quantize_weights": ([i32, i32, p, p, p, p, p], ctypes.c_int),
             "qvae_act_workspace_bytes": ([i64], sz),
             "qvae_act_absmax_quant": ([p, i64, p, p, p, sz, p], ctypes.c_int),
+            "qvae_act_absmax_quant_noalloc": ([p, i64, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
@@ -149,6 +151,13 @@ def qvae_act_absmax_quant(x: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tens
     _check("qvae_act_absmax_quant",
            lib().qvae_act_absmax_quant(_ptr(x), x.numel(), _ptr(xq), _ptr(x_scale), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qvae_act_absmax_quant_noalloc(x: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor,
+                                  stream=None) -> None:
+    """Same as qvae_act_absmax_quant with the library's fixed scratch (no workspace)."""
+    _check("qvae_act_absmax_quant_noalloc",
+           lib().qvae_act_absmax_quant_noalloc(_ptr(x), x.numel(), _ptr(xq), _ptr(x_scale), _stream(stream)))
 
 
 def act_absmax_quant(x: torch.Tensor, stream=None, workspace: Optional[torch.Tensor] = None):
