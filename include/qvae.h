@@ -217,6 +217,17 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  */
 int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode);
 
+/*
+ * Activation-pass override for tuning and tests (process-wide): 0 automatic
+ * (currently two passes, which measured faster), 1 single pass whenever the
+ * tensor fits in one co-resident grid's registers
+ * (about 9.7 M values on a 148-SM B200; each thread holds up to 64 values,
+ * the CTAs exchange partial maxima through a bounded grid barrier in the
+ * workspace, x is read once), 2 always two passes (absmax, then quantise).
+ * Both give identical codes and scale.
+ */
+int qvae_set_act_passes(int32_t mode);
+
 /* The tiling the next convolution of this shape would use: out[0..6] = MS,
  * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2). */
 int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7);

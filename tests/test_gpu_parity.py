@@ -85,8 +85,15 @@ def test_weight_codes_scales_and_packing(q, Cin, Cout):
 
 # -------------------------------------------------------------- activations
 
-def check_act(q, x_dev):
-    xq, s = q.act_absmax_quant(x_dev)
+@pytest.fixture(params=[1, 2], ids=["single-pass", "two-pass"])
+def passes(q, request):
+    q.qvae_set_act_passes(request.param)
+    yield request.param
+    q.qvae_set_act_passes(0)
+
+
+def check_act(q, x_dev, workspace=None):
+    xq, s = q.act_absmax_quant(x_dev, workspace=workspace)
     torch.cuda.synchronize()
     qx, s_ref = oracle.act_quant(dev_bits(x_dev))
     assert np.array_equal(s.cpu().numpy().view(np.uint32), np.array([s_ref]).view(np.uint32))
@@ -96,12 +103,13 @@ def check_act(q, x_dev):
 
 
 @pytest.mark.parametrize("name", ["single_96_64x64", "decoder_top_384_128x128"])
-def test_act_quant_workloads(q, name):
+def test_act_quant_workloads(q, name, passes):
     check_act(q, synth.draw_workload(name)[0].x.cuda())
 
 
-@pytest.mark.parametrize("numel", [1, 7, 8, 15, 16, 17, 1000, 4095, 65537, 1 << 20, 3 * (1 << 20) + 5])
-def test_act_quant_ragged_lengths(q, numel):
+@pytest.mark.parametrize("numel", [1, 7, 8, 15, 16, 17, 1000, 4095, 65537, 1 << 20, 3 * (1 << 20) + 5,
+                                   7_000_003, 9_700_000, 12_000_001])
+def test_act_quant_ragged_lengths(q, numel, passes):
     g = torch.Generator().manual_seed(numel)
     x = (torch.randn(numel, generator=g) * 3).to(torch.bfloat16)
     check_act(q, x.cuda())
@@ -123,7 +131,18 @@ def test_act_quant_every_bf16_value_many_scales(q):
         check_act(q, torch.from_numpy(vals).to(torch.bfloat16).cuda())
 
 
-def test_act_quant_zero_and_empty(q):
+def test_act_quant_shared_workspace_many_calls(q, passes):
+    """The single pass keeps a grid-barrier counter in the workspace: reuse one
+    workspace across calls of different sizes and absmax positions."""
+    ws = torch.empty(q.qvae_act_workspace_bytes(1), dtype=torch.uint8, device="cuda")
+    g = torch.Generator().manual_seed(5)
+    for k, n in enumerate([4096, 6_291_456, 17, 1_000_000, 6_291_456, 333_333]):
+        x = torch.randn(n, generator=g).to(torch.bfloat16)
+        x[(k * 7919) % n] = 20.0 + k
+        check_act(q, x.cuda(), workspace=ws)
+
+
+def test_act_quant_zero_and_empty(q, passes):
     check_act(q, torch.zeros(1000, dtype=torch.bfloat16, device="cuda"))
     x = torch.zeros(0, dtype=torch.bfloat16, device="cuda")
     xq, s = q.act_absmax_quant(x)
@@ -131,7 +150,7 @@ def test_act_quant_zero_and_empty(q):
     assert s.item() == 0.0
 
 
-def test_act_quant_tiny_scales(q):
+def test_act_quant_tiny_scales(q, passes):
     """Subnormal absmax takes the plain-divide branch."""
     vals = np.array([1e-39, -5e-40, 3e-41, 0.0, 2e-39], dtype=np.float32)
     check_act(q, torch.from_numpy(vals).to(torch.bfloat16).cuda())

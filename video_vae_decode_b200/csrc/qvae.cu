@@ -27,6 +27,7 @@ using qvae::ConvArgs;
 thread_local std::string t_last_error;
 uint64_t g_wait_limit_ns = 2000000000ull;
 int32_t g_force[5] = {0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair)
+int g_act_mode = 0;                   // 0 automatic (two passes), 1 single pass when it fits, 2 two passes
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
@@ -383,6 +384,72 @@ int act_grid(int64_t numel, int sms) {
 
 constexpr size_t kActWorkspace = 16384;  // 4096 partial maxima
 
+// Co-resident CTAs of the single-pass quantiser for V vectors per thread (0 if
+// it cannot launch), cached per device.
+int g_fused_blocks[kMaxDevices][5] = {};
+
+template <int V>
+int fused_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qvae::act_absmax_quant_fused_kernel<V>,
+                                                    qvae::kFusedThreads, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int V>
+cudaError_t launch_fused(int grid, cudaStream_t stream, const void* x, int64_t numel, void* ws, int8_t* xq,
+                         float* x_scale) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(qvae::kFusedThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the grid barrier cannot deadlock
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qvae::act_absmax_quant_fused_kernel<V>, static_cast<const uint4*>(x),
+                            numel / 8, static_cast<const uint16_t*>(x), numel, static_cast<uint32_t*>(ws),
+                            reinterpret_cast<uint2*>(xq), xq, x_scale, g_wait_limit_ns * 2);
+}
+
+// Single pass when the tensor fits in one co-resident grid's registers
+// (up to 8 vectors of 8 values per thread); returns false to use two passes.
+bool try_fused_act(int dev, int sms, const void* x, int64_t numel, int8_t* xq, float* x_scale, void* ws,
+                   size_t ws_bytes, cudaStream_t stream, int* rc) {
+  const int64_t nvec = numel / 8;
+  static const int kV[5] = {1, 2, 4, 6, 8};
+  for (int vi = 0; vi < 5; ++vi) {
+    if (g_fused_blocks[dev][vi] == 0) {
+      const int b = vi == 0 ? fused_blocks_per_sm<1>() : vi == 1 ? fused_blocks_per_sm<2>()
+                  : vi == 2 ? fused_blocks_per_sm<4>() : vi == 3 ? fused_blocks_per_sm<6>()
+                  : fused_blocks_per_sm<8>();
+      g_fused_blocks[dev][vi] = b > 0 ? b : -1;
+    }
+    if (g_fused_blocks[dev][vi] < 0) continue;
+    const int64_t max_grid = static_cast<int64_t>(g_fused_blocks[dev][vi]) * sms;
+    const int64_t per_cta = static_cast<int64_t>(qvae::kFusedThreads) * kV[vi];
+    const int64_t grid = std::max<int64_t>(1, ceil_div(nvec, per_cta));
+    if (grid > max_grid) continue;
+    if (16 + 4 * grid > static_cast<int64_t>(ws_bytes)) return false;
+    cudaError_t e = cudaMemsetAsync(ws, 0, 16, stream);  // arrival counter and generation
+    if (e == cudaSuccess) {
+      const int g = static_cast<int>(grid);
+      e = vi == 0 ? launch_fused<1>(g, stream, x, numel, ws, xq, x_scale)
+        : vi == 1 ? launch_fused<2>(g, stream, x, numel, ws, xq, x_scale)
+        : vi == 2 ? launch_fused<4>(g, stream, x, numel, ws, xq, x_scale)
+        : vi == 3 ? launch_fused<6>(g, stream, x, numel, ws, xq, x_scale)
+                  : launch_fused<8>(g, stream, x, numel, ws, xq, x_scale);
+    }
+    *rc = (e == cudaSuccess) ? QVAE_OK : cuda_fail(e, "single-pass activation quantiser launch");
+    return true;
+  }
+  return false;
+}
+
 int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* ws,
                size_t ws_bytes, cudaStream_t stream) {
   if (numel < 0) return QVAE_ERR_ARG;
@@ -397,6 +464,10 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   int dev, sms, rc;
   if ((rc = current_device(&dev))) return rc;
   if ((rc = sm_count(dev, &sms))) return rc;
+  // The single pass reads x once but needs a counter reset and a cooperative
+  // launch; measured slower than two passes at every size here, so it runs only
+  // when asked for.
+  if (g_act_mode == 1 && try_fused_act(dev, sms, x, numel, xq, x_scale, ws, ws_bytes, stream, &rc)) return rc;
   const int g1 = act_grid(numel, sms);
   uint32_t* partial = static_cast<uint32_t*>(ws);
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, stream>>>(
@@ -634,6 +705,12 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
   g_force[2] = SA;
   g_force[3] = SB;
   g_force[4] = mode;
+  return QVAE_OK;
+}
+
+int qvae_set_act_passes(int32_t mode) {
+  if (mode < 0 || mode > 2) return QVAE_ERR_ARG;
+  g_act_mode = mode;
   return QVAE_OK;
 }
 
