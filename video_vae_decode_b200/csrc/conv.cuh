@@ -236,7 +236,15 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------- MMA issuer
+    // Descriptors are built once; every operand start inside the rings is the
+    // base descriptor plus an offset in 16-byte units (all offsets stay inside
+    // the 14-bit start-address field), so each MMA costs a few integer adds.
     const uint32_t idesc = idesc_i8(kPair ? 256 : 128, a.NT);
+    const uint64_t a_desc0 = sw128_kmajor_desc(a_ring, kGroupStride);
+    const uint64_t b_desc0 = sw128_kmajor_desc(b_ring, 1024u);
+    const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
+    const uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
+    const uint32_t ms = static_cast<uint32_t>(a.MS), nt = static_cast<uint32_t>(a.NT);
     uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
     bool issued = false;
     auto commit = [&](uint32_t bar) {
@@ -252,36 +260,40 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       const int nkb = (3 - kt_lo) * a.nchunks;
       if (!mbar_wait(acc_empty + 8 * cs, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
       tc_fence_after();
-      const uint32_t d_tile = tmem_base + cs * static_cast<uint32_t>(a.MS * a.NT);
-      bool first = true;
+      const uint32_t d_tile = tmem_base + cs * ms * nt;
+      uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
       for (int kb = 0; kb < nkb; ++kb) {
         const int ch = kb % a.nchunks;
         if (!mbar_wait(a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
         tc_fence_after();
-        const int ksteps = (ch == a.nchunks - 1) ? a.last_ksteps : 4;
-        const uint32_t a_stage = a_ring + as * a.a_stage_bytes;
+        const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
+        const uint64_t a_stage = a_desc0 + as * a_stage16;
         for (int tap9 = 0; tap9 < 9; ++tap9) {
-          const int kh = tap9 / 3, kw = tap9 % 3;
+          const uint32_t kh = static_cast<uint32_t>(tap9) / 3u, kw = static_cast<uint32_t>(tap9) % 3u;
           if (!mbar_wait(b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
           tc_fence_after();
-          const uint32_t b_stage = b_ring + bs * a.b_stage_bytes;
-          for (int s = 0; s < a.MS; ++s) {
-            // sub-tile s, tap (kh, kw): box row s*16 + kh, column kw
-            const uint32_t a_rows = a_stage + static_cast<uint32_t>(s * kTileRows + kh) * kGroupStride +
-                                    static_cast<uint32_t>(kw) * 128u;
-            for (int k = 0; k < ksteps; ++k) {
-              const uint64_t ad = sw128_kmajor_desc(a_rows + 32u * k, kGroupStride);
-              const uint64_t bd = sw128_kmajor_desc(b_stage + 32u * k, 1024u);
-              const uint32_t acc = (first && k == 0) ? 0u : 1u;
-              if (kPair) {
-                mma_i8_pair(d_tile + static_cast<uint32_t>(s * a.NT), ad, bd, idesc, acc);
-              } else {
-                mma_i8(d_tile + static_cast<uint32_t>(s * a.NT), ad, bd, idesc, acc);
+          // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+          const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+          const uint64_t b_tap = b_desc0 + bs * b_stage16;
+#pragma unroll
+          for (uint32_t s = 0; s < 4; ++s) {
+            if (s < ms) {
+#pragma unroll
+              for (uint32_t k = 0; k < 4; ++k) {
+                if (k < ksteps) {
+                  const uint64_t ad = a_tap + s * sub16 + 2u * k;  // 32 bytes of K = 2 units
+                  const uint64_t bd = b_tap + 2u * k;
+                  if (kPair) {
+                    mma_i8_pair(d_tile + s * nt, ad, bd, idesc, (k == 0) ? acc : 1u);
+                  } else {
+                    mma_i8(d_tile + s * nt, ad, bd, idesc, (k == 0) ? acc : 1u);
+                  }
+                }
               }
-              issued = true;
             }
           }
-          first = false;
+          acc = 1u;
+          issued = true;
           commit(b_empty + 8 * bs);
           if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
         }
