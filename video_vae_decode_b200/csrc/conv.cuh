@@ -75,7 +75,8 @@ struct ConvArgs {
   uint64_t wait_limit_ns;
 };
 
-constexpr int kConvThreads = 192;
+constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
+constexpr int kConvThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
 constexpr int kMaxStages = 12;
 constexpr uint32_t kEpiStageBytes = 4096;  // per epilogue warp: 2 buffers x 32 pixels x 64 B
 
@@ -104,6 +105,93 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvArgs& a, int tile, ui
   return c;
 }
 
+struct MmaRings {
+  uint32_t a_ring, b_ring;                       // shared-memory operand rings
+  uint32_t a_full, a_empty, b_full, b_empty;     // ring barriers
+  uint32_t acc_full, acc_empty;                  // accumulator barriers
+  uint32_t tmem_base;
+};
+
+// MMA issuer (one thread of the pair's leader CTA).  Descriptors are built
+// once; every operand start inside the rings is the base descriptor plus an
+// offset in 16-byte units (all offsets stay inside the 14-bit start-address
+// field), so each MMA costs a few integer adds.  Per tap: kMS sub-tiles, each
+// four k-steps of 32 channels into its own accumulator.  Returns false when a
+// wait gave up (abort or time limit).
+template <bool kPair, int kMS>
+__device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
+                                               volatile int* abort_flag, uint64_t limit, int first_tile,
+                                               int tile_step, uint32_t rank, bool& issued) {
+  const uint32_t idesc = idesc_i8(kPair ? 256 : 128, a.NT);
+  const uint64_t a_desc0 = sw128_kmajor_desc(r.a_ring, kGroupStride);
+  const uint64_t b_desc0 = sw128_kmajor_desc(r.b_ring, 1024u);
+  const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
+  constexpr uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
+  const uint32_t nt = static_cast<uint32_t>(a.NT);
+  uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
+  auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
+    if (kPair) {
+      mma_i8_pair(d, ad, bd, idesc, acc);
+    } else {
+      mma_i8(d, ad, bd, idesc, acc);
+    }
+  };
+  auto commit = [&](uint32_t bar) {
+    if (kPair) {
+      mma_commit_pair_multicast(bar, 0x3);
+    } else {
+      mma_commit(bar);
+    }
+  };
+  for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
+    const TileCoord c = decode_tile<kPair>(a, tile, rank);
+    const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
+    const int nkb = (3 - kt_lo) * a.nchunks;
+    if (!mbar_wait(r.acc_empty + 8 * cs, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
+    tc_fence_after();
+    const uint32_t d_tile = r.tmem_base + cs * static_cast<uint32_t>(kMS) * nt;
+    uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int ch = kb % a.nchunks;
+      if (!mbar_wait(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) return false;
+      tc_fence_after();
+      const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
+      const uint64_t a_stage = a_desc0 + as * a_stage16;
+      for (int tap9 = 0; tap9 < 9; ++tap9) {
+        const uint32_t kh = static_cast<uint32_t>(tap9) / 3u, kw = static_cast<uint32_t>(tap9) % 3u;
+        if (!mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+        const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+        const uint64_t b_tap = b_desc0 + bs * b_stage16;
+        if (ksteps == 4u) {
+#pragma unroll
+          for (int s = 0; s < kMS; ++s) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
+              mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < kMS; ++s) {
+            for (uint32_t k = 0; k < ksteps; ++k)
+              mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+          }
+        }
+        acc = 1u;
+        issued = true;
+        commit(r.b_empty + 8 * bs);
+        if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
+      }
+      commit(r.a_empty + 8 * as);
+      if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
+    }
+    commit(r.acc_full + 8 * cs);
+    if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
+  }
+  return true;
+}
+
 template <bool kAcc32, bool kPair>
 __global__ void __launch_bounds__(kConvThreads, 1)
     conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
@@ -116,7 +204,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
   const uint32_t epi_stage = b_ring + a.SB * a.b_stage_bytes;  // 1024-aligned
-  const uint32_t bars = epi_stage + 4 * kEpiStageBytes;        // 8-byte mbarriers
+  const uint32_t bars = epi_stage + kEpiWarps * kEpiStageBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 16;
@@ -124,7 +212,8 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
   volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
-  float* const epi_smem = reinterpret_cast<float*>(misc + 16);  // 4 warps x 2 x NT floats
+  // NT scales then NT biases, shared by the epilogue warps, 16-byte aligned for vector loads
+  float* const epi_smem = reinterpret_cast<float*>(base_ptr + ((drain_bar + 8 + 16 + 15 - base) & ~15u));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;      // 0 = leader of the pair
@@ -143,7 +232,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, kPair ? 8 : 4);  // one arrive per epilogue warp (of both CTAs)
+      mbar_init(acc_empty + 8 * i, kPair ? 2 * kEpiWarps : kEpiWarps);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -236,75 +325,26 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------- MMA issuer
-    // Descriptors are built once; every operand start inside the rings is the
-    // base descriptor plus an offset in 16-byte units (all offsets stay inside
-    // the 14-bit start-address field), so each MMA costs a few integer adds.
-    const uint32_t idesc = idesc_i8(kPair ? 256 : 128, a.NT);
-    const uint64_t a_desc0 = sw128_kmajor_desc(a_ring, kGroupStride);
-    const uint64_t b_desc0 = sw128_kmajor_desc(b_ring, 1024u);
-    const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
-    const uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
-    const uint32_t ms = static_cast<uint32_t>(a.MS), nt = static_cast<uint32_t>(a.NT);
-    uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
+    // One instantiation per sub-tile count, so that the MMA sequence of a tap
+    // is straight-line code.
+    MmaRings r{a_ring, b_ring, a_full, a_empty, b_full, b_empty, acc_full, acc_empty, tmem_base};
     bool issued = false;
-    auto commit = [&](uint32_t bar) {
-      if (kPair) {
-        mma_commit_pair_multicast(bar, 0x3);
-      } else {
-        mma_commit(bar);
-      }
-    };
-    for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
-      const TileCoord c = decode_tile<kPair>(a, tile, rank);
-      const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
-      const int nkb = (3 - kt_lo) * a.nchunks;
-      if (!mbar_wait(acc_empty + 8 * cs, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
-      tc_fence_after();
-      const uint32_t d_tile = tmem_base + cs * ms * nt;
-      uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int ch = kb % a.nchunks;
-        if (!mbar_wait(a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
-        tc_fence_after();
-        const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
-        const uint64_t a_stage = a_desc0 + as * a_stage16;
-        for (int tap9 = 0; tap9 < 9; ++tap9) {
-          const uint32_t kh = static_cast<uint32_t>(tap9) / 3u, kw = static_cast<uint32_t>(tap9) % 3u;
-          if (!mbar_wait(b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) goto mma_done;
-          tc_fence_after();
-          // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
-          const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
-          const uint64_t b_tap = b_desc0 + bs * b_stage16;
-#pragma unroll
-          for (uint32_t s = 0; s < 4; ++s) {
-            if (s < ms) {
-#pragma unroll
-              for (uint32_t k = 0; k < 4; ++k) {
-                if (k < ksteps) {
-                  const uint64_t ad = a_tap + s * sub16 + 2u * k;  // 32 bytes of K = 2 units
-                  const uint64_t bd = b_tap + 2u * k;
-                  if (kPair) {
-                    mma_i8_pair(d_tile + s * nt, ad, bd, idesc, (k == 0) ? acc : 1u);
-                  } else {
-                    mma_i8(d_tile + s * nt, ad, bd, idesc, (k == 0) ? acc : 1u);
-                  }
-                }
-              }
-            }
-          }
-          acc = 1u;
-          issued = true;
-          commit(b_empty + 8 * bs);
-          if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
-        }
-        commit(a_empty + 8 * as);
-        if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
-      }
-      commit(acc_full + 8 * cs);
-      if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
+    bool ok;
+    switch (a.MS) {
+      case 1:
+        ok = mma_issue_loop<kPair, 1>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+        break;
+      case 2:
+        ok = mma_issue_loop<kPair, 2>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+        break;
+      case 3:
+        ok = mma_issue_loop<kPair, 3>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+        break;
+      default:
+        ok = mma_issue_loop<kPair, 4>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+        break;
     }
-  mma_done:
-    if (*abort_flag && issued) {
+    if (!ok && *abort_flag && issued) {
       // Wait for the tensor cores to finish what was issued before TMEM is freed.
       int dummy = 0;
       if (kPair) {
@@ -316,18 +356,25 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    // Warp q owns TMEM lanes 32q..32q+31 = tile rows 4q..4q+3 x 8 columns.  Each
-    // 32-channel slice is converted, staged in shared memory (64-byte swizzle)
-    // and written by one TMA store of a 32 x 8 x 4 box, which also drops the
-    // rows and columns beyond the image edge.
+    // A warp may read only the TMEM lane quarter warp % 4; lane quarter q holds
+    // tile rows 4q..4q+3 x 8 columns.  Two warps share each quarter: the
+    // tile's (sub-tile, 32-channel slice) items alternate between them.  Each
+    // item is converted, staged in shared memory (64-byte swizzle) and written
+    // by one TMA store of a 32 x 8 x 4 box, which also drops the rows and
+    // columns beyond the image edge.  The TMEM load of a warp's next item is
+    // in flight while the current one is converted.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
-    float* const sc = epi_smem + (warp - 2) * 2 * a.NT;
+    const int nsl = a.NT >> 5;
+    const int items = a.MS * nsl;
+    float* const sc = epi_smem;
     float* const bi = sc + a.NT;
     const uint32_t stage = epi_stage + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;
     const uint32_t empty_leader = kPair ? map_to_cta(acc_empty, 0) : acc_empty;
     uint32_t buf = 0;
     uint32_t cs = 0, cp = 0;
+    int scale_co0 = -1;
     grid_dependency_wait();
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
@@ -336,62 +383,94 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      if (!kAcc32) {
+      if (!kAcc32 && c.co0 != scale_co0) {
+        // every epilogue warp sees the same tiles: refill the shared table
+        // once the previous tile's items are converted
+        named_barrier_sync(1, 32 * kEpiWarps);
         const float sa = *a.x_scale;
-        for (int j = lane; j < a.NT; j += 32) {
+        for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
           sc[j] = __fmul_rn(sa, a.w_scale[c.co0 + j]);
           bi[j] = a.bias ? __bfloat162float(a.bias[c.co0 + j]) : 0.0f;
         }
-        __syncwarp();
+        scale_co0 = c.co0;
+        named_barrier_sync(1, 32 * kEpiWarps);
       }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cs * static_cast<uint32_t>(a.MS * a.NT);
-      for (int s = 0; s < a.MS; ++s) {
-        const int h = c.h0 + s * kTileRows + row / kTileW;
-        const int w = c.w0 + row % kTileW;
-        for (int cc = 0; cc < a.NT; cc += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(s * a.NT + cc), v);
-          tmem_ld_wait();
-          if (kAcc32) {
-            if (h >= a.H || w >= a.W) continue;
+      auto issue = [&](int j, uint32_t(&v)[32]) {
+        const int s = j / nsl;
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(s * a.NT + ((j - s * nsl) << 5)), v);
+      };
+      auto process = [&](int j, const uint32_t(&v)[32]) {
+        const int s = j / nsl;
+        const int cc = (j - s * nsl) << 5;
+        if (kAcc32) {
+          const int h = c.h0 + s * kTileRows + row / kTileW;
+          const int w = c.w0 + row % kTileW;
+          if (h < a.H && w < a.W) {
             const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
             int4* dst = reinterpret_cast<int4*>(a.acc_out + pix * a.Cout + c.co0 + cc);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               dst[e] = make_int4(static_cast<int>(v[4 * e]), static_cast<int>(v[4 * e + 1]),
                                  static_cast<int>(v[4 * e + 2]), static_cast<int>(v[4 * e + 3]));
-          } else {
-            uint32_t packed[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float y0 = __fmul_rn(__int2float_rn(static_cast<int>(v[2 * e])), sc[cc + 2 * e]);
-              float y1 = __fmul_rn(__int2float_rn(static_cast<int>(v[2 * e + 1])), sc[cc + 2 * e + 1]);
-              y0 = __fadd_rn(y0, bi[cc + 2 * e]);
-              y1 = __fadd_rn(y1, bi[cc + 2 * e + 1]);
-              const __nv_bfloat162 p = __floats2bfloat162_rn(y0, y1);
-              packed[e] = *reinterpret_cast<const uint32_t*>(&p);
-            }
-            // the store issued two slices ago read this buffer: let it finish
-            if (lane == 0) bulk_wait_group_read<1>();
-            __syncwarp();
-            const uint32_t line = stage + buf * 2048u + static_cast<uint32_t>(lane) * 64u;
-            const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((k ^ swz) << 4)),
-                           "r"(packed[4 * k]), "r"(packed[4 * k + 1]), "r"(packed[4 * k + 2]),
-                           "r"(packed[4 * k + 3])
-                           : "memory");
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_5d(&tmap_out, stage + buf * 2048u, c.co0 + cc, c.w0,
-                           c.h0 + s * kTileRows + q * 4, c.t, c.n);
-              bulk_commit_group();
-            }
-            buf ^= 1u;
           }
+        } else {
+          const float4* sc4 = reinterpret_cast<const float4*>(sc + cc);
+          const float4* bi4 = reinterpret_cast<const float4*>(bi + cc);
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            // y = float(acc) * scale, rounded, then + bias, rounded: two
+            // channels per packed instruction
+            const float4 f = sc4[e];
+            const float4 b = bi4[e];
+            const uint64_t x01 = f32x2_pack(__int2float_rn(static_cast<int>(v[4 * e])),
+                                            __int2float_rn(static_cast<int>(v[4 * e + 1])));
+            const uint64_t x23 = f32x2_pack(__int2float_rn(static_cast<int>(v[4 * e + 2])),
+                                            __int2float_rn(static_cast<int>(v[4 * e + 3])));
+            const uint64_t y01 = f32x2_add_rn(f32x2_mul_rn(x01, f32x2_pack(f.x, f.y)), f32x2_pack(b.x, b.y));
+            const uint64_t y23 = f32x2_add_rn(f32x2_mul_rn(x23, f32x2_pack(f.z, f.w)), f32x2_pack(b.z, b.w));
+            float y0, y1, y2, y3;
+            f32x2_unpack(y01, y0, y1);
+            f32x2_unpack(y23, y2, y3);
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
+            packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
+            packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+          }
+          // the store issued two items ago read this buffer: let it finish
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          const uint32_t line = stage + buf * 2048u + static_cast<uint32_t>(lane) * 64u;
+          const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((k ^ swz) << 4)),
+                         "r"(packed[4 * k]), "r"(packed[4 * k + 1]), "r"(packed[4 * k + 2]),
+                         "r"(packed[4 * k + 3])
+                         : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_5d(&tmap_out, stage + buf * 2048u, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
+            bulk_commit_group();
+          }
+          buf ^= 1u;
         }
+      };
+      uint32_t va[32], vb[32];
+      int j = half;
+      if (j < items) issue(j, va);
+      while (j < items) {
+        tmem_ld_wait(va);
+        if (j + 2 < items) issue(j + 2, vb);
+        process(j, va);
+        j += 2;
+        if (j >= items) break;
+        tmem_ld_wait(vb);
+        if (j + 2 < items) issue(j + 2, va);
+        process(j, vb);
+        j += 2;
       }
       tc_fence_before();
       __syncwarp();

@@ -94,8 +94,8 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 uint32_t smem_needed(const Tiling& t) {
   const uint32_t bars = 8 * qvae::kMaxStages * 4 + 16 + 16 + 8;
-  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + 4 * qvae::kEpiStageBytes + bars + 16 +
-         4 * 2 * t.NT * 4;
+  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + qvae::kEpiWarps * qvae::kEpiStageBytes + bars +
+         16 + 16 + 2 * t.NT * 4;
 }
 
 // Pipeline depths for a geometry: the deepest weight ring (up to 9 stages,
