@@ -31,6 +31,7 @@ DATASHEET_INT8_TOPS = 4500.0          # B200 dense INT8, NVIDIA datasheet
 INT8_PER_BF16 = 2.0                    # nominal dense INT8 : BF16 ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 10**6
+SPIN_CYCLES = 200_000                  # ~100 us of GPU spin ahead of each event-timed group
 
 
 def parse():
@@ -43,6 +44,8 @@ def parse():
     ap.add_argument("--layer", type=int, default=0, help="layer index inside the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
+                    help="timed steps as CUDA-graph replays (one graph per buffer set) or direct launches")
     return ap.parse_args()
 
 
@@ -251,7 +254,11 @@ def run_ours(args):
     s = layer.shape
     w, b = layer.w.to(dev), layer.bias.to(dev)
     packed0, s_w = qvae.quantize_weights(w)                # once, as at model load
-    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    # A side stream (CUDA graphs cannot capture the legacy default stream);
+    # every launch and copy below runs on it.
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
 
     # Buffer sets (input, codes, output, packed weights) rotate so that every
     # step reads and writes memory that is not in L2, as a decoder layer does:
@@ -274,10 +281,32 @@ def run_ours(args):
     def conv(st):
         qvae.qvae_causal_conv3d_w8a8(st["xq"], st["x_scale"], st["packed"], s_w, b, st["out"], stream)
 
-    for i in range(args.warmup):
-        st = sets[i % n_sets]
+    def step(st):
         act(st)
         conv(st)
+
+    # One CUDA graph per buffer set holds that set's step (the three kernels,
+    # with their programmatic launch dependencies): a replay costs the host one
+    # call, so the timed loop measures the device, not the Python launch path.
+    if args.launch == "graph":
+        step(sets[0])  # first call outside capture: one-time attribute setup
+        torch.cuda.synchronize()
+        graphs = []
+        for st in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(st)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+        def run_step(i):
+            graphs[i % n_sets].replay()
+    else:
+        def run_step(i):
+            step(sets[i % n_sets])
+
+    for i in range(args.warmup):
+        run_step(i)
     torch.cuda.synchronize()
     if qvae.qvae_get_error() != 0:
         raise RuntimeError("device-side timeout during warm-up")
@@ -291,9 +320,7 @@ def run_ours(args):
     with ClockSampler(dev.index) as clk:
         e_start.record(stream)
         for i in range(K):
-            st = sets[i % n_sets]
-            act(st)
-            conv(st)
+            run_step(i)
         e_end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -303,11 +330,14 @@ def run_ours(args):
     if qvae.qvae_get_error() != 0:
         raise RuntimeError("device-side timeout during timing")
 
-    # ---- per-kernel durations (for the roofline): events around each launch
+    # ---- per-kernel durations (for the roofline): events around each launch.
+    # A GPU spin ahead of each group keeps the device behind the host, so the
+    # events time the kernels and not the host's launch gaps.
     R = max(20, min(K, 400))
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
     for i in range(R):
         st = sets[i % n_sets]
+        torch.cuda._sleep(SPIN_CYCLES)
         ev[i][0].record(stream)
         act(st)
         ev[i][1].record(stream)
@@ -357,6 +387,8 @@ def run_ours(args):
                    "tiling": qvae.qvae_get_conv_tiling(s.N, s.T, s.H, s.W, s.Cin, s.Cout),
                    "l2": (f"inputs, codes, outputs and packed weights rotate over {n_sets} buffer sets "
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
+                   "launch": ("one CUDA graph replay per step (act absmax, act quantise, conv)"
+                              if args.launch == "graph" else "direct launches from Python"),
                    "ops_per_layer": ops},
         "ms_per_layer": {"step": ms_per_step, "act_absmax_quant": statistics.mean(act_ms),
                          "conv": conv_mean, "conv_median": statistics.median(conv_ms)},

@@ -1,0 +1,97 @@
+"""The per-layer path (act quantiser + conv, and qvae_decode_layers) inside a CUDA graph.
+
+The library's calls launch on the caller's stream, allocate nothing and never
+synchronise, so a decoder can capture them once and replay.  A replay must
+give bit-identical results to direct calls on the same data, including data
+written into the captured input buffers after the capture.
+"""
+import pytest
+import torch
+
+from video_vae_decode_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from video_vae_decode_b200 import qvae
+    qvae.lib()
+    yield qvae
+
+
+def bits(t):
+    return t.view(torch.int16)
+
+
+def test_layer_step_replays_in_a_cuda_graph(q):
+    s = synth.LayerShape(192, 192, 24, 40, T=2)
+    gen = torch.Generator().manual_seed(21)
+    t0 = synth.draw_layer(gen, s, outliers=True)
+    t1 = synth.draw_layer(gen, s, outliers=False, drift=True)
+    x = t0.x.cuda()
+    w, b = t0.w.cuda(), t0.bias.cuda()
+    packed, s_w = q.quantize_weights(w)
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    sa = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(q.qvae_act_workspace_bytes(x.numel()), dtype=torch.uint8, device="cuda")
+    out = torch.empty((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
+
+    def direct(xin):
+        xq_r, sa_r = q.act_absmax_quant(xin)
+        return q.causal_conv3d_w8a8(xq_r, sa_r, packed, s_w, b, s.Cout), xq_r, sa_r
+
+    ref0, xq0, sa0 = direct(t0.x.cuda())
+    ref1, _, _ = direct(t1.x.cuda())
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        q.qvae_act_absmax_quant(x, xq, sa, ws, stream)
+        q.qvae_causal_conv3d_w8a8(xq, sa, packed, s_w, b, out, stream)
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.qvae_get_error() == 0
+    assert torch.equal(xq, xq0) and torch.equal(sa, sa0)
+    assert torch.equal(bits(out), bits(ref0))
+
+    x.copy_(t1.x.cuda())                                     # new data, same buffers
+    out.fill_(0)
+    torch.cuda.synchronize()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.qvae_get_error() == 0
+    assert torch.equal(bits(out), bits(ref1))
+
+
+def test_decode_layers_replays_in_a_cuda_graph(q):
+    shapes = [synth.LayerShape(96, 192, 20, 24), synth.LayerShape(192, 96, 20, 24)]
+    gen = torch.Generator().manual_seed(22)
+    specs, refs = [], []
+    for s in shapes:
+        t = synth.draw_layer(gen, s, outliers=True)
+        x, w, b = t.x.cuda(), t.w.cuda(), t.bias.cuda()
+        packed, s_w = q.quantize_weights(w)
+        out = torch.zeros((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
+        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=True))
+        xq, s_a = q.act_absmax_quant(x)
+        refs.append(q.causal_conv3d_w8a8(xq, s_a, packed, s_w, b, s.Cout))
+    layers = q.make_layers(specs)
+    ws = torch.empty(q.qvae_decode_workspace_bytes(layers), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        q.qvae_decode_layers(layers, ws, stream)
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.qvae_get_error() == 0
+    for sp, ref in zip(specs, refs):
+        assert torch.equal(bits(sp["out"]), bits(ref))

@@ -129,6 +129,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   constexpr uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
   const uint32_t nt = static_cast<uint32_t>(a.NT);
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
+  bool b_ready = false;  // b_full of stage bs already seen complete
   auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
     if (kPair) {
       mma_i8_pair(d, ad, bd, idesc, acc);
@@ -159,8 +160,15 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
       const uint64_t a_stage = a_desc0 + as * a_stage16;
       for (int tap9 = 0; tap9 < 9; ++tap9) {
         const uint32_t kh = static_cast<uint32_t>(tap9) / 3u, kw = static_cast<uint32_t>(tap9) % 3u;
-        if (!mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
+        if (!b_ready && !mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
         tc_fence_after();
+        {
+          // probe the next weight stage now; its result is used only after this
+          // tap's MMAs are issued, so the probe's latency is hidden behind them
+          const uint32_t nbs = (bs + 1 == static_cast<uint32_t>(a.SB)) ? 0u : bs + 1;
+          const uint32_t nbp = (bs + 1 == static_cast<uint32_t>(a.SB)) ? bp ^ 1u : bp;
+          b_ready = mbar_test_wait(r.b_full + 8 * nbs, nbp);
+        }
         // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
         const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
         const uint64_t b_tap = b_desc0 + bs * b_stage16;

@@ -91,10 +91,14 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* red) {
 // ------------------------------------------------------------ activations
 
 constexpr int kActThreads = 256;
+constexpr int kAbsUnroll = 8;    // 16-byte loads in flight per thread, absmax pass
+constexpr int kQuantUnroll = 4;  // 32-byte (16-value) groups in flight per thread, quantise pass
 
-// Pass 1: per-block absmax (as 15-bit magnitude codes) of a bf16 tensor.  Plain cached
-// loads: when x fits in L2 the second pass reads it from there.
-// x is 16-byte aligned; nvec = numel / 8 full vectors; block 0 also covers the tail.
+// Pass 1: per-block absmax (as 15-bit magnitude codes) of a bf16 tensor.
+// x is 16-byte aligned; nvec = numel / 8 full vectors; block 0 also covers the
+// tail.  Each thread keeps kAbsUnroll loads in flight.  Plain cached loads:
+// the most recently read part of x is still in L2 when pass 2, which walks
+// the tensor backwards, starts.
 __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __restrict__ x,
                                                                   int64_t nvec,
                                                                   const uint16_t* __restrict__ xs,
@@ -102,38 +106,63 @@ __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __
                                                                   uint32_t* __restrict__ partial) {
   __shared__ uint32_t red[kActThreads / 32];
   grid_dependents_launch();  // the quantiser may start its prologue
-  uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+  uint32_t m[4] = {0u, 0u, 0u, 0u};
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
   int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
-  for (; i + 3 * stride < nvec; i += 4 * stride) {
-    const uint4 a = __ldg(x + i), b = __ldg(x + i + stride);
-    const uint4 c = __ldg(x + i + 2 * stride), d = __ldg(x + i + 3 * stride);
-    m0 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m0, a.x), a.y), a.z), a.w);
-    m1 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m1, b.x), b.y), b.z), b.w);
-    m2 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m2, c.x), c.y), c.z), c.w);
-    m3 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m3, d.x), d.y), d.z), d.w);
+  for (; i + (kAbsUnroll - 1) * stride < nvec; i += kAbsUnroll * stride) {
+    uint4 v[kAbsUnroll];
+#pragma unroll
+    for (int u = 0; u < kAbsUnroll; ++u) v[u] = __ldg(x + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kAbsUnroll; ++u)
+      m[u & 3] = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m[u & 3], v[u].x), v[u].y), v[u].z),
+                               v[u].w);
   }
   for (; i < nvec; i += stride) {
     const uint4 a = __ldg(x + i);
-    m0 = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m0, a.x), a.y), a.z), a.w);
+    m[0] = abs_bits_max2(abs_bits_max2(abs_bits_max2(abs_bits_max2(m[0], a.x), a.y), a.z), a.w);
   }
   if (blockIdx.x == 0) {
     for (int64_t k = nvec * 8 + threadIdx.x; k < numel; k += kActThreads)
-      m0 = max(m0, static_cast<uint32_t>(xs[k]) & 0x7FFFu);
+      m[0] = max(m[0], static_cast<uint32_t>(xs[k]) & 0x7FFFu);
   }
-  const uint32_t m = block_max_u32<kActThreads>(max(max(m0, m1), max(m2, m3)), red);
-  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+  const uint32_t mm = block_max_u32<kActThreads>(max(max(m[0], m[1]), max(m[2], m[3])), red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = mm;
+}
+
+// 16 bf16 values (two 16-byte vectors) -> 16 codes (one 16-byte vector).
+__device__ __forceinline__ uint4 quant16(const Quantizer& z, bool zero, const uint4& a, const uint4& b) {
+  if (zero) return make_uint4(0u, 0u, 0u, 0u);
+  return make_uint4(quant4(z, a.x, a.y), quant4(z, a.z, a.w), quant4(z, b.x, b.y), quant4(z, b.z, b.w));
 }
 
 // Pass 2: reduce the partial maxima, derive the scale, write INT8 codes.
-// Pairs of 16-byte bf16 vectors become one 16-byte code vector; nvec2 = numel / 16.
+// Group g (g < nvec2 = numel / 16) is 16 values: two 16-byte bf16 vectors in,
+// one 16-byte code vector out.  Groups are visited from the end of the tensor
+// to its start: the re-read of x begins with what pass 1 read last (still in
+// L2), and the start of xq, which the convolution reads first, is written
+// last.  The first loads of x are issued before waiting for pass 1 (x was
+// complete before pass 1 began).
 __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
     const uint4* __restrict__ x, int64_t nvec2, const uint16_t* __restrict__ xs, int64_t numel,
     const uint32_t* __restrict__ partial, int npartial, uint4* __restrict__ xq,
     int8_t* __restrict__ xq_bytes, float* __restrict__ x_scale) {
   __shared__ uint32_t red[kActThreads / 32];
   grid_dependents_launch();  // the convolution may start its prologue
-  grid_dependency_wait();    // the partial maxima of the previous kernel are complete
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
+  const int64_t last = nvec2 - 1;
+  uint4 va[kQuantUnroll], vb[kQuantUnroll];
+  const bool full = i + (kQuantUnroll - 1) * stride < nvec2;
+  if (full) {
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t g = last - (i + u * stride);
+      va[u] = __ldcs(x + 2 * g);
+      vb[u] = __ldcs(x + 2 * g + 1);
+    }
+  }
+  grid_dependency_wait();  // the partial maxima of the previous kernel are complete
   uint32_t m = 0;
   for (int k = threadIdx.x; k < npartial; k += kActThreads) m = max(m, partial[k]);
   m = block_max_u32<kActThreads>(m, red);
@@ -141,36 +170,29 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
   const float s = __fdiv_rn(amax, 127.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *x_scale = s;
   const Quantizer z = make_quantizer(s);
+  const bool zero = (s == 0.0f);
 
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
-  for (; i + stride < nvec2; i += 2 * stride) {
-    const uint4 a0 = __ldcs(x + 2 * i), a1 = __ldcs(x + 2 * i + 1);
-    const uint4 b0 = __ldcs(x + 2 * (i + stride)), b1 = __ldcs(x + 2 * (i + stride) + 1);
-    uint4 qa, qb;
-    if (s == 0.0f) {
-      qa = make_uint4(0, 0, 0, 0);
-      qb = qa;
-    } else {
-      qa = make_uint4(quant4(z, a0.x, a0.y), quant4(z, a0.z, a0.w), quant4(z, a1.x, a1.y),
-                      quant4(z, a1.z, a1.w));
-      qb = make_uint4(quant4(z, b0.x, b0.y), quant4(z, b0.z, b0.w), quant4(z, b1.x, b1.y),
-                      quant4(z, b1.z, b1.w));
+  if (full) {
+    while (true) {
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) xq[last - (i + u * stride)] = quant16(z, zero, va[u], vb[u]);
+      i += kQuantUnroll * stride;
+      if (i + (kQuantUnroll - 1) * stride >= nvec2) break;
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int64_t g = last - (i + u * stride);
+        va[u] = __ldcs(x + 2 * g);
+        vb[u] = __ldcs(x + 2 * g + 1);
+      }
     }
-    xq[i] = qa;
-    xq[i + stride] = qb;
   }
   for (; i < nvec2; i += stride) {
-    const uint4 a0 = __ldcs(x + 2 * i), a1 = __ldcs(x + 2 * i + 1);
-    uint4 qa = make_uint4(0, 0, 0, 0);
-    if (s != 0.0f)
-      qa = make_uint4(quant4(z, a0.x, a0.y), quant4(z, a0.z, a0.w), quant4(z, a1.x, a1.y),
-                      quant4(z, a1.z, a1.w));
-    xq[i] = qa;
+    const int64_t g = last - i;
+    xq[g] = quant16(z, zero, __ldcs(x + 2 * g), __ldcs(x + 2 * g + 1));
   }
   if (blockIdx.x == 0) {
     for (int64_t k = nvec2 * 16 + threadIdx.x; k < numel; k += kActThreads) {
-      const uint32_t c = (s == 0.0f) ? 0u : z.code_byte(bf16_bits_to_f32(xs[k]));
+      const uint32_t c = zero ? 0u : z.code_byte(bf16_bits_to_f32(xs[k]));
       xq_bytes[k] = static_cast<int8_t>(static_cast<uint8_t>(c));
     }
   }

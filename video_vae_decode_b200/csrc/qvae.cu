@@ -376,10 +376,20 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
 
 // ------------------------------------------------------------- activations
 
+// Blocks of the absmax pass: enough for kAbsUnroll vectors per thread, at
+// most eight 256-thread blocks per SM (full occupancy).
 int act_grid(int64_t numel, int sms) {
   const int64_t vec = numel / 8;
-  const int64_t want = ceil_div(std::max<int64_t>(vec, 1), qvae::kActThreads * 4);
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 4LL * sms)));
+  const int64_t want = ceil_div(std::max<int64_t>(vec, 1), qvae::kActThreads * qvae::kAbsUnroll);
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms)));
+}
+
+// Blocks of the quantise pass: kQuantUnroll 16-value groups per thread, at
+// most eight blocks per SM.
+int quant_grid(int64_t numel, int sms) {
+  const int64_t nvec2 = numel / 16;
+  const int64_t want = ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * qvae::kQuantUnroll);
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms)));
 }
 
 constexpr size_t kActWorkspace = 16384;  // 4096 partial maxima
@@ -474,8 +484,7 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
       static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
-  const int g2 = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>(ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * 2), 4LL * sms)));
+  const int g2 = quant_grid(numel, sms);
   QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, stream, 1,
                              static_cast<const uint4*>(x), nvec2, static_cast<const uint16_t*>(x), numel,
                              static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
@@ -614,8 +623,7 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
       static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, partial);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
-  const int g2 = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>(ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * 2), 4LL * sms)));
+  const int g2 = quant_grid(numel, sms);
   QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, st, 1,
                              static_cast<const uint4*>(x_bf16), nvec2, static_cast<const uint16_t*>(x_bf16),
                              numel, static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
