@@ -212,10 +212,11 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  *   MS    1..4;  NT  a multiple of 32 dividing Cout, <= 256;  MS * NT <= 512
  *   SA/SB activation / weight pipeline stages (<= 12)
  *   mode  1 = one CTA per MMA, 2 = CTA pairs (cta_group::2, M = 256 per MMA)
+ *   G     taps per weight stage: 1, or 3 (one kernel row; MS <= 2)
  * Zero = automatic (a cost model over the shape).  A forced value that
  * cannot be used for a shape makes the convolution return an error.
  */
-int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode);
+int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode, int32_t G);
 
 /*
  * Activation-pass override for tuning and tests (process-wide): 0 automatic
@@ -228,9 +229,9 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
  */
 int qvae_set_act_passes(int32_t mode);
 
-/* The tiling the next convolution of this shape would use: out[0..6] = MS,
- * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2). */
-int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7);
+/* The tiling the next convolution of this shape would use: out[0..7] = MS,
+ * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G. */
+int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out8);
 
 #if defined(__GNUC__)
 #pragma GCC visibility pop

@@ -102,6 +102,7 @@ def test_tiling_choice_is_valid():
         assert 1 <= t["MS"] <= 4 and t["MS"] * t["NT"] <= 512 and t["mode"] in (1, 2)
         assert Cout % t["NT"] == 0 and t["NT"] % 32 == 0 and t["NT"] <= 256
         assert 1 <= t["SA"] <= 12 and 1 <= t["SB"] <= 12
+        assert t["G"] == 1 or (t["G"] == 3 and t["MS"] <= 2)
         assert t["acc_buffers"] == (2 if 2 * t["MS"] * t["NT"] <= 512 else 1)
         rows = 16 * t["MS"] * t["mode"]
         tiles = N * T * -(-H // rows) * -(-W // 8) * (Cout // t["NT"])
@@ -110,6 +111,9 @@ def test_tiling_choice_is_valid():
     try:
         t = qvae.qvae_get_conv_tiling(1, 1, 100, 100, 128, 128)
         assert (t["MS"], t["NT"], t["SA"], t["SB"], t["mode"]) == (1, 64, 2, 3, 1)
+        qvae.qvae_set_conv_tiling(MS=1, NT=192, mode=2, G=3)
+        t = qvae.qvae_get_conv_tiling(1, 1, 100, 100, 192, 192)
+        assert (t["MS"], t["NT"], t["mode"], t["G"]) == (1, 192, 2, 3)
     finally:
         qvae.qvae_set_conv_tiling()
     with pytest.raises(qvae.QvaeError):
@@ -120,3 +124,7 @@ def test_tiling_choice_is_valid():
         qvae.qvae_set_conv_tiling(MS=3, NT=256)
     with pytest.raises(qvae.QvaeError):
         qvae.qvae_set_conv_tiling(mode=3)
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(G=2)
+    with pytest.raises(qvae.QvaeError):
+        qvae.qvae_set_conv_tiling(MS=3, G=3)

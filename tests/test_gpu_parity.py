@@ -184,7 +184,9 @@ TILINGS = [None,
            dict(mode=1), dict(mode=1, MS=1), dict(mode=1, MS=3), dict(mode=1, MS=4, NT=64, SA=1, SB=2),
            dict(mode=1, MS=1, SA=1, SB=1), dict(mode=1, NT=32),
            dict(mode=2), dict(mode=2, MS=1), dict(mode=2, MS=2), dict(mode=2, MS=3), dict(mode=2, MS=4),
-           dict(mode=2, MS=1, SA=1, SB=1), dict(mode=2, NT=32), dict(mode=2, MS=2, NT=64, SA=2, SB=9)]
+           dict(mode=2, MS=1, SA=1, SB=1), dict(mode=2, NT=32), dict(mode=2, MS=2, NT=64, SA=2, SB=9),
+           dict(mode=1, MS=1, G=3), dict(mode=1, MS=2, G=3, SA=1, SB=1), dict(mode=2, MS=1, G=3),
+           dict(mode=2, MS=2, NT=32, G=3, SA=2, SB=2), dict(mode=2, MS=1, G=3, SA=1, SB=1)]
 
 
 @pytest.mark.parametrize("tiling", TILINGS)

@@ -49,6 +49,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace qvae {
@@ -64,9 +66,11 @@ struct ConvArgs {
   int tiles_w, tiles_h, tiles_n, num_tiles;  // tiles_h counts CTA-pair row bands in pair mode
   int nchunks, last_ksteps;   // 128-channel chunks; 32-channel k-steps in the last one
   int SA, SB, acc_stages;     // pipeline depths
+  int G;                      // taps per weight stage (1 or 3; 9 / G stages per 128-channel chunk)
   uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
   uint32_t a_box_bytes;       // bytes one activation box delivers
-  uint32_t b_stage_bytes;     // weight rows this CTA loads per tap x 128 B
+  uint32_t b_tap_bytes;       // weight rows this CTA loads per tap x 128 B
+  uint32_t b_stage_bytes;     // G x b_tap_bytes
   uint32_t tmem_cols;
   const float* x_scale;       // device scalar
   const float* w_scale;       // [Cout]
@@ -115,10 +119,11 @@ struct MmaRings {
 // MMA issuer (one thread of the pair's leader CTA).  Descriptors are built
 // once; every operand start inside the rings is the base descriptor plus an
 // offset in 16-byte units (all offsets stay inside the 14-bit start-address
-// field), so each MMA costs a few integer adds.  Per tap: kMS sub-tiles, each
-// four k-steps of 32 channels into its own accumulator.  Returns false when a
-// wait gave up (abort or time limit).
-template <bool kPair, int kMS>
+// field), so each MMA costs a few integer adds.  A weight stage holds kG
+// taps; per tap: kMS sub-tiles, each four k-steps of 32 channels into its own
+// accumulator.  One wait and one commit per stage.  Returns false when a wait
+// gave up (abort or time limit).
+template <bool kPair, int kMS, int kG>
 __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
                                                volatile int* abort_flag, uint64_t limit, int first_tile,
                                                int tile_step, uint32_t rank, bool& issued) {
@@ -126,6 +131,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   const uint64_t a_desc0 = sw128_kmajor_desc(r.a_ring, kGroupStride);
   const uint64_t b_desc0 = sw128_kmajor_desc(r.b_ring, 1024u);
   const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
+  const uint32_t b_tap16 = a.b_tap_bytes >> 4;
   constexpr uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
   const uint32_t nt = static_cast<uint32_t>(a.NT);
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
@@ -158,35 +164,40 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
       tc_fence_after();
       const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
       const uint64_t a_stage = a_desc0 + as * a_stage16;
-      for (int tap9 = 0; tap9 < 9; ++tap9) {
-        const uint32_t kh = static_cast<uint32_t>(tap9) / 3u, kw = static_cast<uint32_t>(tap9) % 3u;
+      for (int grp = 0; grp < 9 / kG; ++grp) {
         if (!b_ready && !mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
         tc_fence_after();
         {
           // probe the next weight stage now; its result is used only after this
-          // tap's MMAs are issued, so the probe's latency is hidden behind them
+          // stage's MMAs are issued, so the probe's latency is hidden behind them
           const uint32_t nbs = (bs + 1 == static_cast<uint32_t>(a.SB)) ? 0u : bs + 1;
           const uint32_t nbp = (bs + 1 == static_cast<uint32_t>(a.SB)) ? bp ^ 1u : bp;
           b_ready = mbar_test_wait(r.b_full + 8 * nbs, nbp);
         }
-        // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
-        const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
-        const uint64_t b_tap = b_desc0 + bs * b_stage16;
-        if (ksteps == 4u) {
+        const uint64_t b_stage = b_desc0 + bs * b_stage16;
 #pragma unroll
-          for (int s = 0; s < kMS; ++s) {
+        for (int g = 0; g < kG; ++g) {
+          const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+          const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+          // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+          const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+          const uint64_t b_tap = b_stage + g * b_tap16;
+          if (ksteps == 4u) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
-              mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+            for (int s = 0; s < kMS; ++s) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
+                mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+            }
+          } else {
+#pragma unroll
+            for (int s = 0; s < kMS; ++s) {
+              for (uint32_t k = 0; k < ksteps; ++k)
+                mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+            }
           }
-        } else {
-#pragma unroll
-          for (int s = 0; s < kMS; ++s) {
-            for (uint32_t k = 0; k < ksteps; ++k)
-              mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
-          }
+          acc = 1u;
         }
-        acc = 1u;
         issued = true;
         commit(r.b_empty + 8 * bs);
         if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
@@ -229,6 +240,12 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   const int first_tile = kPair ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
   const int tile_step = kPair ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
 
+  // Start the tensor-map descriptor fetches before anything else.
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+  }
+  if (threadIdx.x == 64 && !kAcc32) prefetch_tmap(&tmap_out);
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.SA; ++i) {
       mbar_init(a_full + 8 * i, 1);
@@ -267,22 +284,24 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     // ------------------------------------------------------------ producer
     // Weights do not depend on the preceding kernel: the first weight stages
     // are filled before waiting for the activation codes.
-    prefetch_tmap(&tmap_x);
-    prefetch_tmap(&tmap_w);
     uint32_t as = 0, ap = 0, bs = 0, bp = 0;
     uint32_t a_armed = 0, a_par = 0, b_armed = 0, b_par = 0;  // per-stage bitmasks
     const uint32_t tx_mult = kPair ? 2u : 1u;                 // bytes both CTAs deliver
     int preissued = 0;
-    auto load_b = [&](const TileCoord& c, int kt, int ch, int tap9) -> bool {
+    const int ngrp = 9 / a.G;  // weight stages per 128-channel chunk
+    auto load_b = [&](const TileCoord& c, int kt, int ch, int grp) -> bool {
       if (!mbar_wait(b_empty + 8 * bs, bp ^ 1, abort_flag, limit, kErrTimeoutProducer)) return false;
-      const int tap = kt * 9 + tap9;  // (kt * 3 + kh) * 3 + kw
-      const int row = (tap * a.nchunks + ch) * a.Cout + c.co0 + static_cast<int>(rank) * (a.NT / 2);
       const uint32_t bar = b_full + 8 * bs;
       if (leader) mbar_arrive_expect_tx(bar, a.b_stage_bytes * tx_mult);
-      if (kPair) {
-        tma_load_2d_pair(b_ring + bs * a.b_stage_bytes, &tmap_w, map_to_cta(bar, 0), 0, row);
-      } else {
-        tma_load_2d(b_ring + bs * a.b_stage_bytes, &tmap_w, bar, 0, row);
+      for (int g = 0; g < a.G; ++g) {
+        const int tap = kt * 9 + grp * a.G + g;  // (kt * 3 + kh) * 3 + kw
+        const int row = (tap * a.nchunks + ch) * a.Cout + c.co0 + static_cast<int>(rank) * (a.NT / 2);
+        const uint32_t dst = b_ring + bs * a.b_stage_bytes + static_cast<uint32_t>(g) * a.b_tap_bytes;
+        if (kPair) {
+          tma_load_2d_pair(dst, &tmap_w, map_to_cta(bar, 0), 0, row);
+        } else {
+          tma_load_2d(dst, &tmap_w, bar, 0, row);
+        }
       }
       b_armed |= 1u << bs;
       b_par = (b_par & ~(1u << bs)) | (bp << bs);
@@ -297,7 +316,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         const int kt = kt_lo + kb / a.nchunks, ch = kb % a.nchunks;
         if (!waited) {
-          for (; preissued < a.SB && preissued < 9; ++preissued)
+          for (; preissued < a.SB && preissued < ngrp; ++preissued)
             if (!load_b(c, kt, ch, preissued)) goto producer_done;
           grid_dependency_wait();
           waited = true;
@@ -317,7 +336,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         a_armed |= 1u << as;
         a_par = (a_par & ~(1u << as)) | (ap << as);
         if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
-        for (int i = preissued; i < 9; ++i)
+        for (int i = preissued; i < ngrp; ++i)
           if (!load_b(c, kt, ch, i)) goto producer_done;
         preissued = 0;
       }
@@ -333,23 +352,35 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------- MMA issuer
-    // One instantiation per sub-tile count, so that the MMA sequence of a tap
-    // is straight-line code.
+    // One instantiation per (sub-tile count, taps per stage), so that the
+    // MMA sequence of a stage is straight-line code.
     MmaRings r{a_ring, b_ring, a_full, a_empty, b_full, b_empty, acc_full, acc_empty, tmem_base};
     bool issued = false;
     bool ok;
-    switch (a.MS) {
-      case 1:
-        ok = mma_issue_loop<kPair, 1>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+    auto run = [&](auto ms, auto g) {
+      return mma_issue_loop<kPair, decltype(ms)::value, decltype(g)::value>(a, r, abort_flag, limit, first_tile,
+                                                                           tile_step, rank, issued);
+    };
+    using G1 = std::integral_constant<int, 1>;
+    using G3 = std::integral_constant<int, 3>;
+    switch (a.MS * 4 + a.G) {
+      case 1 * 4 + 3:
+        ok = run(std::integral_constant<int, 1>{}, G3{});
         break;
-      case 2:
-        ok = mma_issue_loop<kPair, 2>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+      case 2 * 4 + 3:
+        ok = run(std::integral_constant<int, 2>{}, G3{});
         break;
-      case 3:
-        ok = mma_issue_loop<kPair, 3>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+      case 1 * 4 + 1:
+        ok = run(std::integral_constant<int, 1>{}, G1{});
+        break;
+      case 2 * 4 + 1:
+        ok = run(std::integral_constant<int, 2>{}, G1{});
+        break;
+      case 3 * 4 + 1:
+        ok = run(std::integral_constant<int, 3>{}, G1{});
         break;
       default:
-        ok = mma_issue_loop<kPair, 4>(a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
+        ok = run(std::integral_constant<int, 4>{}, G1{});
         break;
     }
     if (!ok && *abort_flag && issued) {
@@ -383,7 +414,22 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     uint32_t buf = 0;
     uint32_t cs = 0, cp = 0;
     int scale_co0 = -1;
-    grid_dependency_wait();
+    // Scale and bias table for output channels co0..co0+NT-1.  Every epilogue
+    // warp sees the same tiles, so all of them take part; the first barrier
+    // lets the previous tile's items finish reading the old table.
+    auto fill_table = [&](int co0) {
+      named_barrier_sync(1, 32 * kEpiWarps);
+      const float sa = *a.x_scale;
+      for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
+        sc[j] = __fmul_rn(sa, a.w_scale[co0 + j]);
+        bi[j] = a.bias ? __bfloat162float(a.bias[co0 + j]) : 0.0f;
+      }
+      scale_co0 = co0;
+      named_barrier_sync(1, 32 * kEpiWarps);
+    };
+    grid_dependency_wait();  // the activation scale is final
+    // the first tile's table is ready before its accumulators are
+    if (!kAcc32 && first_tile < a.num_tiles) fill_table(decode_tile<kPair>(a, first_tile, rank).co0);
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
       int ok = 1;
@@ -391,18 +437,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      if (!kAcc32 && c.co0 != scale_co0) {
-        // every epilogue warp sees the same tiles: refill the shared table
-        // once the previous tile's items are converted
-        named_barrier_sync(1, 32 * kEpiWarps);
-        const float sa = *a.x_scale;
-        for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
-          sc[j] = __fmul_rn(sa, a.w_scale[c.co0 + j]);
-          bi[j] = a.bias ? __bfloat162float(a.bias[c.co0 + j]) : 0.0f;
-        }
-        scale_co0 = c.co0;
-        named_barrier_sync(1, 32 * kEpiWarps);
-      }
+      if (!kAcc32 && c.co0 != scale_co0) fill_table(c.co0);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cs * static_cast<uint32_t>(a.MS * a.NT);
       auto issue = [&](int j, uint32_t(&v)[32]) {
         const int s = j / nsl;

@@ -26,7 +26,7 @@ using qvae::ConvArgs;
 
 thread_local std::string t_last_error;
 uint64_t g_wait_limit_ns = 2000000000ull;
-int32_t g_force[5] = {0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair)
+int32_t g_force[6] = {0, 0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair), G
 int g_act_mode = 0;                   // 0 automatic (two passes), 1 single pass when it fits, 2 two passes
 
 constexpr int kMaxDevices = 64;
@@ -84,8 +84,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 struct Tiling {
   bool pair;
-  int MS, NT, SA, SB, acc_stages;
-  uint32_t a_stage_bytes, a_box_bytes, b_stage_bytes, tmem_cols, smem_bytes;
+  int MS, NT, SA, SB, acc_stages, G;
+  uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
   int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
   double est_cycles;
 };
@@ -98,8 +98,8 @@ uint32_t smem_needed(const Tiling& t) {
          16 + 16 + 2 * t.NT * 4;
 }
 
-// Pipeline depths for a geometry: the deepest weight ring (up to 9 stages,
-// one tap each) next to two activation stages, else the best that fits.
+// Pipeline depths for a geometry: the deepest weight ring (up to 9 stages of
+// G taps each) next to two activation stages, else the best that fits.
 bool fit_stages(Tiling* t) {
   if (g_force[2] || g_force[3]) {
     t->SA = g_force[2] ? g_force[2] : 2;
@@ -115,11 +115,12 @@ bool fit_stages(Tiling* t) {
 }
 
 // Relative cost of a geometry on `sms` SMs, in SM cycles: waves x the time of
-// a CTA tile.  A tile is its weight stages (one per tap and 128-channel chunk),
-// each MS x k-steps MMAs of 128 x NT x 32 at the measured cycles per MMA for
-// that N plus a measured ~330-cycle handshake, and the epilogue when the
-// accumulator cannot be double-buffered.  A CTA pair shares weight loads but
-// measured no faster than single CTAs here, so it is charged slightly more.
+// a CTA tile.  A tile is its weight stages (G taps of one 128-channel chunk
+// each), each tap MS x k-steps MMAs of 128 x NT x 32 at the measured cycles
+// per MMA for that N, plus a handshake per stage, an exposed activation load
+// per chunk when the activation ring has one stage, and the epilogue when the
+// accumulator cannot be double-buffered.  CTA pairs load half the weights per
+// SM and measured 2-4 % faster than single CTAs of the same geometry.
 double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   double taps_t = 0;
   for (int64_t f = 0; f < std::min<int64_t>(s.T, 2); ++f) taps_t += static_cast<double>(f + 1);
@@ -129,23 +130,27 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   const double mma = std::max(0.52 * t.NT + 8.0, 60.0 + 0.17 * t.NT);
   const int nchunks = (s.Cin + 127) / 128;
   const double ksteps_total = s.Cin / 32.0;
-  const double stages = taps_t * 9.0 * nchunks;
+  const double stages = taps_t * 9.0 / t.G * nchunks;
   const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 330.0 + 1500.0 +
+                          (t.SA == 1 ? 1500.0 * taps_t * nchunks : 0.0) +
                           (t.acc_stages == 1 ? 6.0 * t.MS * t.NT : 0.0);
   const double slots = t.pair ? std::floor(sms / 2.0) : sms;
   const double waves = std::ceil(static_cast<double>(t.num_tiles) / slots);
-  return (waves * per_tile + (t.acc_stages == 1 ? 0.0 : 6.0 * t.MS * t.NT)) * (t.pair ? 1.05 : 1.0);
+  return (waves * per_tile + (t.acc_stages == 1 ? 0.0 : 6.0 * t.MS * t.NT)) * (t.pair ? 0.98 : 1.0);
 }
 
-int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, Tiling* t) {
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, Tiling* t) {
+  if (G != 1 && !(G == 3 && MS <= 2)) return QVAE_ERR_ARG;  // kernel instantiations
   t->pair = pair;
   t->MS = MS;
   t->NT = NT;
+  t->G = G;
   t->ctas_per_tile = pair ? 2 : 1;
   const int rows = MS * qvae::kTileRows + 2;
   t->a_box_bytes = static_cast<uint32_t>(rows) * qvae::kGroupStride;
   t->a_stage_bytes = (t->a_box_bytes + 1023u) & ~1023u;
-  t->b_stage_bytes = static_cast<uint32_t>(pair ? NT / 2 : NT) * 128u;
+  t->b_tap_bytes = static_cast<uint32_t>(pair ? NT / 2 : NT) * 128u;
+  t->b_stage_bytes = static_cast<uint32_t>(G) * t->b_tap_bytes;
   const int acc_cols = MS * NT;
   if (acc_cols > 512) return QVAE_ERR_ARG;
   t->acc_stages = (2 * acc_cols <= 512) ? 2 : 1;
@@ -172,12 +177,15 @@ int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148) {
       for (int nt = 32; nt <= std::min(256, s.Cout); nt += 32) {
         if (s.Cout % nt) continue;
         if (g_force[1] && nt != g_force[1]) continue;
-        Tiling u;
-        if (make_geometry(s, mode == 2, ms, nt, &u) != QVAE_OK) continue;
-        u.est_cycles = estimate_cycles(s, u, sms);
-        if (!found || u.est_cycles < t->est_cycles) {
-          *t = u;
-          found = true;
+        for (int g = 1; g <= 3; g += 2) {
+          if (g_force[5] && g != g_force[5]) continue;
+          Tiling u;
+          if (make_geometry(s, mode == 2, ms, nt, g, &u) != QVAE_OK) continue;
+          u.est_cycles = estimate_cycles(s, u, sms);
+          if (!found || u.est_cycles < t->est_cycles) {
+            *t = u;
+            found = true;
+          }
         }
       }
     }
@@ -330,6 +338,8 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.acc_stages = t.acc_stages;
   a.a_stage_bytes = t.a_stage_bytes;
   a.a_box_bytes = t.a_box_bytes;
+  a.G = t.G;
+  a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
   a.x_scale = x_scale;
@@ -702,17 +712,20 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return QVAE_OK;
 }
 
-int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode) {
+int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode, int32_t G) {
   if (MS < 0 || MS > 4) return QVAE_ERR_ARG;
   if (NT && (NT % 32 || NT > 256 || NT < 32)) return QVAE_ERR_ARG;
   if (MS && NT && MS * NT > 512) return QVAE_ERR_ARG;
   if (SA < 0 || SA > qvae::kMaxStages || SB < 0 || SB > qvae::kMaxStages) return QVAE_ERR_ARG;
   if (mode < 0 || mode > 2) return QVAE_ERR_ARG;
+  if (G != 0 && G != 1 && G != 3) return QVAE_ERR_ARG;
+  if (G == 3 && MS > 2) return QVAE_ERR_ARG;
   g_force[0] = MS;
   g_force[1] = NT;
   g_force[2] = SA;
   g_force[3] = SB;
   g_force[4] = mode;
+  g_force[5] = G;
   return QVAE_OK;
 }
 
@@ -722,8 +735,8 @@ int qvae_set_act_passes(int32_t mode) {
   return QVAE_OK;
 }
 
-int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7) {
-  if (!out7) return QVAE_ERR_ARG;
+int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out8) {
+  if (!out8) return QVAE_ERR_ARG;
   int rc = check_shape(shape);
   if (rc) return rc;
   int sms = 148, dev;
@@ -731,13 +744,14 @@ int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out7) {
   cudaGetLastError();
   Tiling t;
   if ((rc = make_tiling(*shape, &t, sms))) return rc;
-  out7[0] = t.MS;
-  out7[1] = t.NT;
-  out7[2] = t.SA;
-  out7[3] = t.SB;
-  out7[4] = t.acc_stages;
-  out7[5] = t.num_tiles * t.ctas_per_tile;
-  out7[6] = t.pair ? 2 : 1;
+  out8[0] = t.MS;
+  out8[1] = t.NT;
+  out8[2] = t.SA;
+  out8[3] = t.SB;
+  out8[4] = t.acc_stages;
+  out8[5] = t.num_tiles * t.ctas_per_tile;
+  out8[6] = t.pair ? 2 : 1;
+  out8[7] = t.G;
   return QVAE_OK;
 }
 

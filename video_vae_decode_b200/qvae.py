@@ -75,7 +75,7 @@ def lib():
             "qvae_get_error": ([p], ctypes.c_int),
             "qvae_set_wait_limit_ns": ([u64], ctypes.c_int),
             "qvae_selftest_wait_timeout": ([u64, p], ctypes.c_int),
-            "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32], ctypes.c_int),
+            "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
             "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), ctypes.POINTER(i32)], ctypes.c_int),
             "qvae_set_act_passes": ([i32], ctypes.c_int),
         }
@@ -244,8 +244,8 @@ def qvae_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("qvae_selftest_wait_timeout", lib().qvae_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
-def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0) -> None:
-    _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(MS, NT, SA, SB, mode))
+def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0, G=0) -> None:
+    _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(MS, NT, SA, SB, mode, G))
 
 
 def qvae_set_act_passes(mode: int = 0) -> None:
@@ -254,6 +254,6 @@ def qvae_set_act_passes(mode: int = 0) -> None:
 
 def qvae_get_conv_tiling(N, T, H, W, Cin, Cout) -> dict:
     shp = make_shape(N, T, H, W, Cin, Cout)
-    out = (ctypes.c_int32 * 7)()
+    out = (ctypes.c_int32 * 8)()
     _check("qvae_get_conv_tiling", lib().qvae_get_conv_tiling(ctypes.byref(shp), out))
-    return dict(zip(("MS", "NT", "SA", "SB", "acc_buffers", "ctas", "mode"), list(out)))
+    return dict(zip(("MS", "NT", "SA", "SB", "acc_buffers", "ctas", "mode", "G"), list(out)))
