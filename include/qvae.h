@@ -219,6 +219,13 @@ int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t mode, int32_t G);
 
 /*
+ * Cap on the number of convolution CTAs (process-wide, tests and tuning):
+ * 0 = the default, one CTA (or CTA pair) per SM up to the number of tiles.
+ * A small cap makes each CTA walk several tiles of a small problem.
+ */
+int qvae_set_conv_cta_limit(int32_t max_ctas);
+
+/*
  * Activation-pass override for tuning and tests (process-wide): 0 automatic
  * (currently two passes, which measured faster), 1 single pass whenever the
  * tensor fits in one co-resident grid's registers

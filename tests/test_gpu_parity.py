@@ -189,11 +189,44 @@ TILINGS = [None,
            dict(mode=2, MS=2, NT=32, G=3, SA=2, SB=2), dict(mode=2, MS=1, G=3, SA=1, SB=1)]
 
 
+@pytest.mark.parametrize("tiling", [dict(mode=1, MS=1), dict(mode=2, MS=1, G=3), dict(mode=1, MS=4, NT=64)])
+def test_conv_few_ctas_many_tiles_exact(q, tiling):
+    # three CTAs (one pair in mode 2) walk all tiles: accumulator buffers and
+    # ring phases wrap many times
+    q.qvae_set_conv_cta_limit(3)
+    try:
+        assert conv_case(q, synth.LayerShape(64, 64, 19, 37, T=4), seed=2, tiling=tiling) == 1.0
+    finally:
+        q.qvae_set_conv_cta_limit(0)
+
+
 @pytest.mark.parametrize("tiling", TILINGS)
 def test_conv_tilings_exact(q, tiling):
     # spans several tiles in h, w and channels, with ragged edges and T > 2
     exact = conv_case(q, synth.LayerShape(64, 64, 19, 37, T=4), seed=1, tiling=tiling)
     assert exact == 1.0
+
+
+# One accumulator buffer of several sub-tiles, handed to the epilogue one by
+# one (the first and last chunk of a tile issued sub-tile by sub-tile): CTA
+# pairs with 3- and 1-tap weight stages, single CTAs with 3 and 4 sub-tiles.
+SPLIT_TILINGS = [dict(mode=2, MS=2, NT=192, G=3, SA=2, SB=3), dict(mode=2, MS=2, NT=192, G=1, SA=2, SB=9),
+                 dict(mode=1, MS=3, NT=96, G=1, SA=1, SB=9), dict(mode=1, MS=4, NT=96, G=1, SA=1, SB=9)]
+
+
+@pytest.mark.parametrize("tiling", SPLIT_TILINGS)
+@pytest.mark.parametrize("shape", [
+    synth.LayerShape(192, 192, 37, 21, T=3),          # 2 chunks (128 + 64): 2, 4 and 6 chunks per tile
+    synth.LayerShape(128, 192, 20, 24, T=2),          # 1 chunk: first and last chunk coincide at t = 0
+])
+@pytest.mark.parametrize("ctas", [0, 4])
+def test_conv_subtile_handoff_exact(q, tiling, shape, ctas):
+    # ctas = 4: every CTA walks several tiles, so hand-offs cross tile boundaries
+    q.qvae_set_conv_cta_limit(ctas)
+    try:
+        assert conv_case(q, shape, seed=5, tiling=tiling, outliers=True) == 1.0
+    finally:
+        q.qvae_set_conv_cta_limit(0)
 
 
 @pytest.mark.parametrize("shape", [

@@ -67,6 +67,7 @@ struct ConvArgs {
   int nchunks, last_ksteps;   // 128-channel chunks; 32-channel k-steps in the last one
   int SA, SB, acc_stages;     // pipeline depths
   int G;                      // taps per weight stage (1 or 3; 9 / G stages per 128-channel chunk)
+  int split;                  // per-sub-tile accumulator hand-off (one accumulator buffer, MS >= 2, SB >= 9 / G)
   uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
   uint32_t a_box_bytes;       // bytes one activation box delivers
   uint32_t b_tap_bytes;       // weight rows this CTA loads per tap x 128 B
@@ -82,7 +83,8 @@ struct ConvArgs {
 constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
 constexpr int kConvThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
 constexpr int kMaxStages = 12;
-constexpr uint32_t kEpiStageBytes = 4096;  // per epilogue warp: 2 buffers x 32 pixels x 64 B
+constexpr uint32_t kEpiStageBytes = 2048;  // per epilogue warp: 32 pixels x 64 B
+constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
 
 struct TileCoord {
   int n, t, h0, w0, co0;
@@ -121,8 +123,15 @@ struct MmaRings {
 // offset in 16-byte units (all offsets stay inside the 14-bit start-address
 // field), so each MMA costs a few integer adds.  A weight stage holds kG
 // taps; per tap: kMS sub-tiles, each four k-steps of 32 channels into its own
-// accumulator.  One wait and one commit per stage.  Returns false when a wait
-// gave up (abort or time limit).
+// accumulator.  One wait and one commit per stage.
+//
+// Accumulator barriers are per (buffer, sub-tile).  With a single buffer
+// (split mode) the first and the last 128-channel chunk of a tile are issued
+// sub-tile by sub-tile over all of the chunk's weight stages, which the ring
+// holds at once: sub-tile s of the last chunk completes (and its epilogue
+// starts) while the later sub-tiles still run, and sub-tile s of the next
+// tile starts as soon as its epilogue has released it.  Returns false when a
+// wait gave up (abort or time limit).
 template <bool kPair, int kMS, int kG>
 __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
                                                volatile int* abort_flag, uint64_t limit, int first_tile,
@@ -133,7 +142,10 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
   const uint32_t b_tap16 = a.b_tap_bytes >> 4;
   constexpr uint32_t sub16 = (kTileRows * kGroupStride) >> 4;  // one 16-row sub-tile
+  constexpr int kGrp = 9 / kG;                                  // weight stages per chunk
   const uint32_t nt = static_cast<uint32_t>(a.NT);
+  const uint32_t sb = static_cast<uint32_t>(a.SB);
+  const bool split = a.split != 0;
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
   bool b_ready = false;  // b_full of stage bs already seen complete
   auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
@@ -150,13 +162,28 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
       mma_commit(bar);
     }
   };
+  // the MMAs of one tap for sub-tile s
+  auto tap_mmas = [&](uint32_t d, uint64_t a_tap, uint64_t b_tap, uint32_t ksteps, uint32_t acc) {
+    if (ksteps == 4u) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
+        mma(d, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+    } else {
+      for (uint32_t k = 0; k < ksteps; ++k) mma(d, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+    }
+  };
   for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
     const TileCoord c = decode_tile<kPair>(a, tile, rank);
     const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
     const int nkb = (3 - kt_lo) * a.nchunks;
-    if (!mbar_wait(r.acc_empty + 8 * cs, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
-    tc_fence_after();
     const uint32_t d_tile = r.tmem_base + cs * static_cast<uint32_t>(kMS) * nt;
+    const uint32_t accb = cs * static_cast<uint32_t>(kMS);  // this buffer's first barrier index
+    if (!split) {
+#pragma unroll
+      for (int s = 0; s < kMS; ++s)
+        if (!mbar_wait(r.acc_empty + 8 * (accb + s), cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
+      tc_fence_after();
+    }
     uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
     for (int kb = 0; kb < nkb; ++kb) {
       const int ch = kb % a.nchunks;
@@ -164,48 +191,90 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
       tc_fence_after();
       const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
       const uint64_t a_stage = a_desc0 + as * a_stage16;
-      for (int grp = 0; grp < 9 / kG; ++grp) {
-        if (!b_ready && !mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
-        tc_fence_after();
-        {
-          // probe the next weight stage now; its result is used only after this
-          // stage's MMAs are issued, so the probe's latency is hidden behind them
-          const uint32_t nbs = (bs + 1 == static_cast<uint32_t>(a.SB)) ? 0u : bs + 1;
-          const uint32_t nbp = (bs + 1 == static_cast<uint32_t>(a.SB)) ? bp ^ 1u : bp;
-          b_ready = mbar_test_wait(r.b_full + 8 * nbs, nbp);
-        }
-        const uint64_t b_stage = b_desc0 + bs * b_stage16;
+      const bool first = kb == 0, last = kb == nkb - 1;
+      if (split && (first || last)) {
+        // sub-tile by sub-tile over the chunk's kGrp stages (all resident)
+        uint32_t st = bs, sp = bp;
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-          const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
-          const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
-          // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
-          const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
-          const uint64_t b_tap = b_stage + g * b_tap16;
-          if (ksteps == 4u) {
-#pragma unroll
-            for (int s = 0; s < kMS; ++s) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
-                mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
-            }
-          } else {
-#pragma unroll
-            for (int s = 0; s < kMS; ++s) {
-              for (uint32_t k = 0; k < ksteps; ++k)
-                mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
-            }
+        for (int s = 0; s < kMS; ++s) {
+          if (first) {
+            if (!mbar_wait(r.acc_empty + 8 * s, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
+            tc_fence_after();
           }
-          acc = 1u;
+          uint32_t acc_s = first ? 0u : 1u;
+          st = bs;
+          sp = bp;
+          for (int grp = 0; grp < kGrp; ++grp) {
+            if (s == 0) {
+              if (!mbar_wait(r.b_full + 8 * st, sp, abort_flag, limit, kErrTimeoutMma)) return false;
+              tc_fence_after();
+            }
+            const uint64_t b_stage = b_desc0 + st * b_stage16;
+#pragma unroll
+            for (int g = 0; g < kG; ++g) {
+              const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+              const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+              const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4) + s * sub16;
+              tap_mmas(d_tile + s * nt, a_tap, b_stage + g * b_tap16, ksteps, acc_s);
+              acc_s = 1u;
+            }
+            issued = true;
+            if (s == kMS - 1) commit(r.b_empty + 8 * st);
+            if (++st == sb) { st = 0; sp ^= 1; }
+          }
+          if (last) commit(r.acc_full + 8 * s);
         }
-        issued = true;
-        commit(r.b_empty + 8 * bs);
-        if (++bs == static_cast<uint32_t>(a.SB)) { bs = 0; bp ^= 1; }
+        bs = st;
+        bp = sp;
+        b_ready = false;
+        acc = 1u;
+      } else {
+        for (int grp = 0; grp < kGrp; ++grp) {
+          if (!b_ready && !mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
+          tc_fence_after();
+          {
+            // probe the next weight stage now; its result is used only after this
+            // stage's MMAs are issued, so the probe's latency is hidden behind them
+            const uint32_t nbs = (bs + 1 == sb) ? 0u : bs + 1;
+            const uint32_t nbp = (bs + 1 == sb) ? bp ^ 1u : bp;
+            b_ready = mbar_test_wait(r.b_full + 8 * nbs, nbp);
+          }
+          const uint64_t b_stage = b_desc0 + bs * b_stage16;
+#pragma unroll
+          for (int g = 0; g < kG; ++g) {
+            const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+            const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+            // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+            const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+            const uint64_t b_tap = b_stage + g * b_tap16;
+            if (ksteps == 4u) {
+#pragma unroll
+              for (int s = 0; s < kMS; ++s) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
+                  mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+              }
+            } else {
+#pragma unroll
+              for (int s = 0; s < kMS; ++s) {
+                for (uint32_t k = 0; k < ksteps; ++k)
+                  mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+              }
+            }
+            acc = 1u;
+          }
+          issued = true;
+          commit(r.b_empty + 8 * bs);
+          if (++bs == sb) { bs = 0; bp ^= 1; }
+        }
       }
       commit(r.a_empty + 8 * as);
       if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
     }
-    commit(r.acc_full + 8 * cs);
+    if (!split) {
+#pragma unroll
+      for (int s = 0; s < kMS; ++s) commit(r.acc_full + 8 * (accb + s));
+    }
     if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
   }
   return true;
@@ -226,8 +295,8 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   const uint32_t bars = epi_stage + kEpiWarps * kEpiStageBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
-  const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 16;
-  const uint32_t drain_bar = acc_empty + 16;
+  const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 8 * kAccBars;
+  const uint32_t drain_bar = acc_empty + 8 * kAccBars;
   uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
   volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -255,7 +324,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       mbar_init(b_full + 8 * i, 1);
       mbar_init(b_empty + 8 * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBars; ++i) {
       mbar_init(acc_full + 8 * i, 1);
       mbar_init(acc_empty + 8 * i, kPair ? 2 * kEpiWarps : kEpiWarps);  // one arrive per epilogue warp (of both CTAs)
     }
@@ -396,27 +465,28 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // A warp may read only the TMEM lane quarter warp % 4; lane quarter q holds
-    // tile rows 4q..4q+3 x 8 columns.  Two warps share each quarter: the
-    // tile's (sub-tile, 32-channel slice) items alternate between them.  Each
-    // item is converted, staged in shared memory (64-byte swizzle) and written
-    // by one TMA store of a 32 x 8 x 4 box, which also drops the rows and
-    // columns beyond the image edge.  The TMEM load of a warp's next item is
-    // in flight while the current one is converted.
+    // tile rows 4q..4q+3 x 8 columns.  Two warps share each quarter: a
+    // sub-tile's 32-channel slices alternate between them.  Sub-tiles are
+    // taken in order, each as soon as its accumulator is complete, and handed
+    // back to the MMA issuer when read.  Each slice is converted, staged in
+    // shared memory (64-byte swizzle) and written by one TMA store of a
+    // 32 x 8 x 4 box, which also drops the rows and columns beyond the image
+    // edge.  The TMEM load of a warp's next slice is in flight while the
+    // current one is converted.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int nsl = a.NT >> 5;
-    const int items = a.MS * nsl;
     float* const sc = epi_smem;
     float* const bi = sc + a.NT;
     const uint32_t stage = epi_stage + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;
     const uint32_t empty_leader = kPair ? map_to_cta(acc_empty, 0) : acc_empty;
-    uint32_t buf = 0;
     uint32_t cs = 0, cp = 0;
     int scale_co0 = -1;
+    bool dead = false;  // a wait gave up: keep pace with the other warps' table barriers, do no work
     // Scale and bias table for output channels co0..co0+NT-1.  Every epilogue
     // warp sees the same tiles, so all of them take part; the first barrier
-    // lets the previous tile's items finish reading the old table.
+    // lets the previous tile's slices finish reading the old table.
     auto fill_table = [&](int co0) {
       named_barrier_sync(1, 32 * kEpiWarps);
       const float sa = *a.x_scale;
@@ -428,100 +498,98 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       named_barrier_sync(1, 32 * kEpiWarps);
     };
     grid_dependency_wait();  // the activation scale is final
-    // the first tile's table is ready before its accumulators are
-    if (!kAcc32 && first_tile < a.num_tiles) fill_table(decode_tile<kPair>(a, first_tile, rank).co0);
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(acc_full + 8 * cs, cp, abort_flag, limit, kErrTimeoutEpilogue);
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      if (!kAcc32 && c.co0 != scale_co0) fill_table(c.co0);
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cs * static_cast<uint32_t>(a.MS * a.NT);
-      auto issue = [&](int j, uint32_t(&v)[32]) {
-        const int s = j / nsl;
-        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(s * a.NT + ((j - s * nsl) << 5)), v);
-      };
-      auto process = [&](int j, const uint32_t(&v)[32]) {
-        const int s = j / nsl;
-        const int cc = (j - s * nsl) << 5;
-        if (kAcc32) {
-          const int h = c.h0 + s * kTileRows + row / kTileW;
-          const int w = c.w0 + row % kTileW;
-          if (h < a.H && w < a.W) {
-            const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
-            int4* dst = reinterpret_cast<int4*>(a.acc_out + pix * a.Cout + c.co0 + cc);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_int4(static_cast<int>(v[4 * e]), static_cast<int>(v[4 * e + 1]),
-                                 static_cast<int>(v[4 * e + 2]), static_cast<int>(v[4 * e + 3]));
-          }
-        } else {
-          const float4* sc4 = reinterpret_cast<const float4*>(sc + cc);
-          const float4* bi4 = reinterpret_cast<const float4*>(bi + cc);
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            // y = float(acc) * scale, rounded, then + bias, rounded: two
-            // channels per packed instruction
-            const float4 f = sc4[e];
-            const float4 b = bi4[e];
-            const uint64_t x01 = f32x2_pack(__int2float_rn(static_cast<int>(v[4 * e])),
-                                            __int2float_rn(static_cast<int>(v[4 * e + 1])));
-            const uint64_t x23 = f32x2_pack(__int2float_rn(static_cast<int>(v[4 * e + 2])),
-                                            __int2float_rn(static_cast<int>(v[4 * e + 3])));
-            const uint64_t y01 = f32x2_add_rn(f32x2_mul_rn(x01, f32x2_pack(f.x, f.y)), f32x2_pack(b.x, b.y));
-            const uint64_t y23 = f32x2_add_rn(f32x2_mul_rn(x23, f32x2_pack(f.z, f.w)), f32x2_pack(b.z, b.w));
-            float y0, y1, y2, y3;
-            f32x2_unpack(y01, y0, y1);
-            f32x2_unpack(y23, y2, y3);
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
-            const __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
-            packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
-            packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
-          }
-          // the store issued two items ago read this buffer: let it finish
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-          const uint32_t line = stage + buf * 2048u + static_cast<uint32_t>(lane) * 64u;
-          const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((k ^ swz) << 4)),
-                         "r"(packed[4 * k]), "r"(packed[4 * k + 1]), "r"(packed[4 * k + 2]),
-                         "r"(packed[4 * k + 3])
-                         : "memory");
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_5d(&tmap_out, stage + buf * 2048u, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
-            bulk_commit_group();
-          }
-          buf ^= 1u;
+      if (!kAcc32 && c.co0 != scale_co0) fill_table(c.co0);  // before the accumulators are ready
+      const uint32_t accb = cs * static_cast<uint32_t>(a.MS);
+      const uint32_t t_buf = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + accb * static_cast<uint32_t>(a.NT);
+      for (int s = 0; s < a.MS && !dead; ++s) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(acc_full + 8 * (accb + s), cp, abort_flag, limit, kErrTimeoutEpilogue);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) {
+          dead = true;
+          break;
         }
-      };
-      uint32_t va[32], vb[32];
-      int j = half;
-      if (j < items) issue(j, va);
-      while (j < items) {
-        tmem_ld_wait(va);
-        if (j + 2 < items) issue(j + 2, vb);
-        process(j, va);
-        j += 2;
-        if (j >= items) break;
-        tmem_ld_wait(vb);
-        if (j + 2 < items) issue(j + 2, va);
-        process(j, vb);
-        j += 2;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (kPair) {
-          mbar_arrive_cluster(empty_leader + 8 * cs);
-        } else {
-          mbar_arrive(acc_empty + 8 * cs);
+        tc_fence_after();
+        const uint32_t t_sub = t_buf + static_cast<uint32_t>(s * a.NT);
+        auto issue = [&](int jj, uint32_t(&v)[32]) { tmem_ld_32x32b_x32(t_sub + static_cast<uint32_t>(jj << 5), v); };
+        auto process = [&](int jj, const uint32_t(&v)[32]) {
+          const int cc = jj << 5;
+          if (kAcc32) {
+            const int h = c.h0 + s * kTileRows + row / kTileW;
+            const int w = c.w0 + row % kTileW;
+            if (h < a.H && w < a.W) {
+              const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
+              int4* dst = reinterpret_cast<int4*>(a.acc_out + pix * a.Cout + c.co0 + cc);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_int4(static_cast<int>(v[4 * e]), static_cast<int>(v[4 * e + 1]),
+                                   static_cast<int>(v[4 * e + 2]), static_cast<int>(v[4 * e + 3]));
+            }
+          } else {
+            const float4* sc4 = reinterpret_cast<const float4*>(sc + cc);
+            const float4* bi4 = reinterpret_cast<const float4*>(bi + cc);
+            uint32_t packed[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              // y = float(acc) * scale, rounded, then + bias, rounded.  The
+              // scalar _rn intrinsics are never contracted into an FMA (packed
+              // f32x2 multiply + add were: one rounding instead of two).
+              const float4 f = sc4[e];
+              const float4 b = bi4[e];
+              const float y0 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e])), f.x), b.x);
+              const float y1 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 1])), f.y), b.y);
+              const float y2 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 2])), f.z), b.z);
+              const float y3 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 3])), f.w), b.w);
+              const __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
+              const __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
+              packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
+              packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+            }
+            // the previous store read this buffer: let it finish
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            const uint32_t line = stage + static_cast<uint32_t>(lane) * 64u;
+            const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((k ^ swz) << 4)),
+                           "r"(packed[4 * k]), "r"(packed[4 * k + 1]), "r"(packed[4 * k + 2]),
+                           "r"(packed[4 * k + 3])
+                           : "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_5d(&tmap_out, stage, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
+              bulk_commit_group();
+            }
+          }
+        };
+        uint32_t va[32], vb[32];
+        // this warp's slices of the sub-tile: jj = j0, j0 + 2, ... (the two
+        // warps of a quarter alternate over the tile's slices in order)
+        int jj = (half + s * nsl) & 1;
+        if (jj < nsl) issue(jj, va);
+        while (jj < nsl) {
+          tmem_ld_wait(va);
+          if (jj + 2 < nsl) issue(jj + 2, vb);
+          process(jj, va);
+          jj += 2;
+          if (jj >= nsl) break;
+          tmem_ld_wait(vb);
+          if (jj + 2 < nsl) issue(jj + 2, va);
+          process(jj, vb);
+          jj += 2;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair) {
+            mbar_arrive_cluster(empty_leader + 8 * (accb + s));
+          } else {
+            mbar_arrive(acc_empty + 8 * (accb + s));
+          }
         }
       }
       if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }

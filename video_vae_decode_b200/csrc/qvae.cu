@@ -27,6 +27,7 @@ using qvae::ConvArgs;
 thread_local std::string t_last_error;
 uint64_t g_wait_limit_ns = 2000000000ull;
 int32_t g_force[6] = {0, 0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair), G
+int32_t g_cta_limit = 0;                  // cap on the conv grid (0 = one CTA per SM); tests and tuning
 int g_act_mode = 0;                   // 0 automatic (two passes), 1 single pass when it fits, 2 two passes
 
 constexpr int kMaxDevices = 64;
@@ -85,6 +86,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 struct Tiling {
   bool pair;
   int MS, NT, SA, SB, acc_stages, G;
+  bool split;  // per-sub-tile accumulator hand-off
   uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
   int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
   double est_cycles;
@@ -93,7 +95,7 @@ struct Tiling {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 uint32_t smem_needed(const Tiling& t) {
-  const uint32_t bars = 8 * qvae::kMaxStages * 4 + 16 + 16 + 8;
+  const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 8;
   return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + qvae::kEpiWarps * qvae::kEpiStageBytes + bars +
          16 + 16 + 2 * t.NT * 4;
 }
@@ -119,7 +121,8 @@ bool fit_stages(Tiling* t) {
 // each), each tap MS x k-steps MMAs of 128 x NT x 32 at the measured cycles
 // per MMA for that N, plus a handshake per stage, an exposed activation load
 // per chunk when the activation ring has one stage, and the epilogue when the
-// accumulator cannot be double-buffered.  CTA pairs load half the weights per
+// accumulator has one buffer and its sub-tiles cannot be handed over one by
+// one.  CTA pairs load half the weights per
 // SM and measured 2-4 % faster than single CTAs of the same geometry.
 double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   double taps_t = 0;
@@ -133,10 +136,12 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   const double stages = taps_t * 9.0 / t.G * nchunks;
   const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 330.0 + 1500.0 +
                           (t.SA == 1 ? 1500.0 * taps_t * nchunks : 0.0) +
-                          (t.acc_stages == 1 ? 6.0 * t.MS * t.NT : 0.0);
+                          (t.acc_stages == 1 && !t.split ? 6.0 * t.MS * t.NT : 0.0);
   const double slots = t.pair ? std::floor(sms / 2.0) : sms;
   const double waves = std::ceil(static_cast<double>(t.num_tiles) / slots);
-  return (waves * per_tile + (t.acc_stages == 1 ? 0.0 : 6.0 * t.MS * t.NT)) * (t.pair ? 0.98 : 1.0);
+  // the last tile's epilogue (its last sub-tile's when they are handed over one by one)
+  const double tail = t.acc_stages == 2 ? 6.0 * t.MS * t.NT : (t.split ? 6.0 * t.NT : 0.0);
+  return (waves * per_tile + tail) * (t.pair ? 0.98 : 1.0);
 }
 
 int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, Tiling* t) {
@@ -159,6 +164,9 @@ int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, Tiling*
   t->tmem_cols = cols;
   if (!fit_stages(t)) return QVAE_ERR_UNSUPPORTED;
   t->smem_bytes = smem_needed(*t);
+  // one accumulator buffer of several sub-tiles: hand them over one by one
+  // when the ring holds a whole chunk's weight stages
+  t->split = t->acc_stages == 1 && MS >= 2 && t->SB >= 9 / G;
   t->tiles_w = static_cast<int>(ceil_div(s.W, qvae::kTileW));
   t->tiles_h = static_cast<int>(ceil_div(s.H, MS * qvae::kTileRows * t->ctas_per_tile));
   t->tiles_n = s.Cout / NT;
@@ -339,6 +347,7 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.a_stage_bytes = t.a_stage_bytes;
   a.a_box_bytes = t.a_box_bytes;
   a.G = t.G;
+  a.split = t.split ? 1 : 0;
   a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
@@ -375,9 +384,12 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
       QVAE_CUDA(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg));
       g_max_clusters[dev] = std::max(n, 1);
     }
-    grid = 2 * std::min(t.num_tiles, g_max_clusters[dev]);
+    int clusters = std::min(t.num_tiles, g_max_clusters[dev]);
+    if (g_cta_limit > 0) clusters = std::max(1, std::min(clusters, g_cta_limit / 2));
+    grid = 2 * clusters;
   } else {
     grid = std::min(t.num_tiles, sms);
+    if (g_cta_limit > 0) grid = std::min(grid, g_cta_limit);
   }
   QVAE_CUDA(launch_dependent(kernel, grid, qvae::kConvThreads, t.smem_bytes, stream, t.pair ? 2 : 1, tmap_x,
                              tmap_w, tmap_out, a));
@@ -726,6 +738,12 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
   g_force[3] = SB;
   g_force[4] = mode;
   g_force[5] = G;
+  return QVAE_OK;
+}
+
+int qvae_set_conv_cta_limit(int32_t max_ctas) {
+  if (max_ctas < 0) return QVAE_ERR_ARG;
+  g_cta_limit = max_ctas;
   return QVAE_OK;
 }
 

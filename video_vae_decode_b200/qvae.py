@@ -26,7 +26,7 @@ EXPORTS = (
     "qvae_quantize_weights", "qvae_act_workspace_bytes", "qvae_act_absmax_quant",
     "qvae_causal_conv3d_w8a8", "qvae_causal_conv3d_w8a8_acc32", "qvae_decode_workspace_bytes",
     "qvae_decode_layers", "qvae_get_error", "qvae_set_wait_limit_ns",
-    "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling",
+    "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
     "qvae_act_absmax_quant_noalloc", "qvae_set_act_passes",
 )
 
@@ -76,6 +76,7 @@ def lib():
             "qvae_set_wait_limit_ns": ([u64], ctypes.c_int),
             "qvae_selftest_wait_timeout": ([u64, p], ctypes.c_int),
             "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
+            "qvae_set_conv_cta_limit": ([i32], ctypes.c_int),
             "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), ctypes.POINTER(i32)], ctypes.c_int),
             "qvae_set_act_passes": ([i32], ctypes.c_int),
         }
@@ -246,6 +247,10 @@ def qvae_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
 
 def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0, G=0) -> None:
     _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(MS, NT, SA, SB, mode, G))
+
+
+def qvae_set_conv_cta_limit(max_ctas: int = 0) -> None:
+    _check("qvae_set_conv_cta_limit", lib().qvae_set_conv_cta_limit(int(max_ctas)))
 
 
 def qvae_set_act_passes(mode: int = 0) -> None:
