@@ -134,7 +134,7 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   const int nchunks = (s.Cin + 127) / 128;
   const double ksteps_total = s.Cin / 32.0;
   const double stages = taps_t * 9.0 / t.G * nchunks;
-  const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 330.0 + 1500.0 +
+  const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 250.0 + 500.0 +
                           (t.SA == 1 ? 1500.0 * taps_t * nchunks : 0.0) +
                           (t.acc_stages == 1 && !t.split ? 6.0 * t.MS * t.NT : 0.0);
   const double slots = t.pair ? std::floor(sms / 2.0) : sms;
