@@ -68,6 +68,7 @@ struct ConvArgs {
   int SA, SB, acc_stages;     // pipeline depths
   int G;                      // taps per weight stage (1 or 3; 9 / G stages per 128-channel chunk)
   int split;                  // per-sub-tile accumulator hand-off (one accumulator buffer, MS >= 2, SB >= 9 / G)
+  int epi_bufs;               // staging buffers per epilogue warp (1 or 2)
   uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
   uint32_t a_box_bytes;       // bytes one activation box delivers
   uint32_t b_tap_bytes;       // weight rows this CTA loads per tap x 128 B
@@ -83,7 +84,7 @@ struct ConvArgs {
 constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
 constexpr int kConvThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
 constexpr int kMaxStages = 12;
-constexpr uint32_t kEpiStageBytes = 2048;  // per epilogue warp: 32 pixels x 64 B
+constexpr uint32_t kEpiBufBytes = 2048;    // one epilogue staging buffer: 32 pixels x 64 B
 constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
 
 struct TileCoord {
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
   const uint32_t epi_stage = b_ring + a.SB * a.b_stage_bytes;  // 1024-aligned
-  const uint32_t bars = epi_stage + kEpiWarps * kEpiStageBytes;  // 8-byte mbarriers
+  const uint32_t bars = epi_stage + kEpiWarps * a.epi_bufs * kEpiBufBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 8 * kAccBars;
@@ -469,9 +470,9 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     // sub-tile's 32-channel slices alternate between them.  Sub-tiles are
     // taken in order, each as soon as its accumulator is complete, and handed
     // back to the MMA issuer when read.  Each slice is converted, staged in
-    // shared memory (64-byte swizzle) and written by one TMA store of a
-    // 32 x 8 x 4 box, which also drops the rows and columns beyond the image
-    // edge.  The TMEM load of a warp's next slice is in flight while the
+    // shared memory (64-byte swizzle; one or two buffers per warp) and written
+    // by one TMA store of a 32 x 8 x 4 box, which also drops the rows and
+    // columns beyond the image edge.  The TMEM load of a warp's next slice is in flight while the
     // current one is converted.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
@@ -479,7 +480,8 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     const int nsl = a.NT >> 5;
     float* const sc = epi_smem;
     float* const bi = sc + a.NT;
-    const uint32_t stage = epi_stage + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;
+    const uint32_t stage = epi_stage + static_cast<uint32_t>((warp - 2) * a.epi_bufs) * kEpiBufBytes;
+    uint32_t buf = 0;
     const uint32_t empty_leader = kPair ? map_to_cta(acc_empty, 0) : acc_empty;
     uint32_t cs = 0, cp = 0;
     int scale_co0 = -1;
@@ -547,10 +549,17 @@ __global__ void __launch_bounds__(kConvThreads, 1)
               packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
               packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
             }
-            // the previous store read this buffer: let it finish
-            if (lane == 0) bulk_wait_group_read<0>();
+            // the store issued epi_bufs slices ago read this buffer: let it finish
+            if (lane == 0) {
+              if (a.epi_bufs == 2) {
+                bulk_wait_group_read<1>();
+              } else {
+                bulk_wait_group_read<0>();
+              }
+            }
             __syncwarp();
-            const uint32_t line = stage + static_cast<uint32_t>(lane) * 64u;
+            const uint32_t sbuf = stage + buf * kEpiBufBytes;
+            const uint32_t line = sbuf + static_cast<uint32_t>(lane) * 64u;
             const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -561,9 +570,10 @@ __global__ void __launch_bounds__(kConvThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_5d(&tmap_out, stage, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
+              tma_store_5d(&tmap_out, sbuf, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
               bulk_commit_group();
             }
+            if (a.epi_bufs == 2) buf ^= 1u;
           }
         };
         uint32_t va[32], vb[32];

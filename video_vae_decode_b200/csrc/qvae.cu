@@ -86,7 +86,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 struct Tiling {
   bool pair;
   int MS, NT, SA, SB, acc_stages, G;
-  bool split;  // per-sub-tile accumulator hand-off
+  bool split;    // per-sub-tile accumulator hand-off
+  int epi_bufs;  // epilogue staging buffers per warp
   uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
   int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
   double est_cycles;
@@ -96,22 +97,34 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 uint32_t smem_needed(const Tiling& t) {
   const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 8;
-  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + qvae::kEpiWarps * qvae::kEpiStageBytes + bars +
+  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + qvae::kEpiWarps * t.epi_bufs * qvae::kEpiBufBytes +
+         bars +
          16 + 16 + 2 * t.NT * 4;
 }
 
 // Pipeline depths for a geometry: the deepest weight ring (up to 9 stages of
-// G taps each) next to two activation stages, else the best that fits.
-bool fit_stages(Tiling* t) {
+// G taps each) next to two activation stages and two epilogue staging
+// buffers per warp, else the best that fits.  `want_sb`: a weight ring depth
+// to reach first with one staging buffer if it does not fit with two (the
+// sub-tile hand-off needs a whole chunk's stages).
+bool fit_stages(Tiling* t, int want_sb = 0) {
   if (g_force[2] || g_force[3]) {
     t->SA = g_force[2] ? g_force[2] : 2;
     t->SB = g_force[3] ? g_force[3] : 4;
-    return smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit);
+    for (t->epi_bufs = 2; t->epi_bufs >= 1; --t->epi_bufs)
+      if (smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit)) return true;
+    return false;
   }
   for (int sa = 2; sa >= 1; --sa) {
     t->SA = sa;
-    for (t->SB = 9; t->SB >= 2; --t->SB)
-      if (smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit)) return true;
+    for (int bufs = 2; bufs >= 1; --bufs) {
+      t->epi_bufs = bufs;
+      for (t->SB = 9; t->SB >= 2; --t->SB) {
+        if (smem_needed(*t) > static_cast<uint32_t>(kSmemLimit)) continue;
+        if (bufs == 2 && want_sb && t->SB < want_sb) break;  // try one staging buffer
+        return true;
+      }
+    }
   }
   return false;
 }
@@ -144,7 +157,7 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   return (waves * per_tile + tail) * (t.pair ? 0.98 : 1.0);
 }
 
-int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, Tiling* t) {
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t) {
   if (G != 1 && !(G == 3 && MS <= 2)) return QVAE_ERR_ARG;  // kernel instantiations
   t->pair = pair;
   t->MS = MS;
@@ -162,17 +175,21 @@ int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, Tiling*
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(t->acc_stages * acc_cols)) cols <<= 1;
   t->tmem_cols = cols;
-  if (!fit_stages(t)) return QVAE_ERR_UNSUPPORTED;
-  t->smem_bytes = smem_needed(*t);
-  // one accumulator buffer of several sub-tiles: hand them over one by one
-  // when the ring holds a whole chunk's weight stages
-  t->split = t->acc_stages == 1 && MS >= 2 && t->SB >= 9 / G;
   t->tiles_w = static_cast<int>(ceil_div(s.W, qvae::kTileW));
   t->tiles_h = static_cast<int>(ceil_div(s.H, MS * qvae::kTileRows * t->ctas_per_tile));
   t->tiles_n = s.Cout / NT;
   const int64_t tiles = s.N * s.T * t->tiles_h * static_cast<int64_t>(t->tiles_w) * t->tiles_n;
   if (tiles > INT32_MAX / 2) return QVAE_ERR_SHAPE;
   t->num_tiles = static_cast<int>(tiles);
+  // One accumulator buffer of several sub-tiles: hand them over one by one
+  // when the weight ring holds a whole chunk's stages.  The hand-off pays
+  // when CTAs walk several tiles; with about one tile per CTA two staging
+  // buffers per epilogue warp (a faster last epilogue) measured better.
+  const int slots = pair ? std::max(1, sms / 2) : std::max(1, sms);
+  const bool want_split = t->acc_stages == 1 && MS >= 2 && 2 * t->num_tiles >= 3 * slots;
+  if (!fit_stages(t, want_split ? 9 / G : 0)) return QVAE_ERR_UNSUPPORTED;
+  t->smem_bytes = smem_needed(*t);
+  t->split = t->acc_stages == 1 && MS >= 2 && t->SB >= 9 / G;
   return QVAE_OK;
 }
 
@@ -188,7 +205,7 @@ int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148) {
         for (int g = 1; g <= 3; g += 2) {
           if (g_force[5] && g != g_force[5]) continue;
           Tiling u;
-          if (make_geometry(s, mode == 2, ms, nt, g, &u) != QVAE_OK) continue;
+          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u) != QVAE_OK) continue;
           u.est_cycles = estimate_cycles(s, u, sms);
           if (!found || u.est_cycles < t->est_cycles) {
             *t = u;
@@ -348,6 +365,7 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.a_box_bytes = t.a_box_bytes;
   a.G = t.G;
   a.split = t.split ? 1 : 0;
+  a.epi_bufs = t.epi_bufs;
   a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
