@@ -38,6 +38,8 @@ def lib():
         L.oracle_act_quant.restype = ctypes.c_int
         L.oracle_conv_acc.argtypes = [p, p, i64, i64, i64, i64, i32, i32, p]
         L.oracle_conv_acc.restype = ctypes.c_int
+        L.oracle_conv_acc_carry.argtypes = [p, p, i64, i64, i64, i64, i32, i32, p]
+        L.oracle_conv_acc_carry.restype = ctypes.c_int
         L.oracle_conv_acc_points.argtypes = [p, p, i64, i64, i64, i64, i32, i32, p, i64, p]
         L.oracle_conv_acc_points.restype = ctypes.c_int
         L.oracle_epilogue.argtypes = [p, i64, i32, f32, p, p, p]
@@ -112,6 +114,22 @@ def conv_acc(qx, qw):
     return acc
 
 
+def conv_acc_carry(qx_ext, qw):
+    """Exact INT32 conv of a streamed chunk. qx_ext int8 [N,T+2,H,W,Cin] whose first
+    two frames are the previous chunk's last two input frames; returns [N,T,H,W,Cout]."""
+    qx_ext = np.ascontiguousarray(qx_ext, dtype=np.int8)
+    qw = np.ascontiguousarray(qw, dtype=np.int8)
+    N, T2, H, W, Cin = qx_ext.shape
+    T = T2 - 2
+    assert T >= 1, "a chunk needs at least one frame after the two carried ones"
+    Cout = qw.shape[0]
+    assert qw.shape == (Cout, Cin, 3, 3, 3)
+    acc = np.empty((N, T, H, W, Cout), dtype=np.int32)
+    _check(lib().oracle_conv_acc_carry(_ptr(qx_ext), _ptr(qw), N, T, H, W, Cin, Cout, _ptr(acc)),
+           "conv_acc_carry")
+    return acc
+
+
 def conv_acc_points(qx, qw, pts):
     """INT32 accumulators at selected pixels. pts int64 [P, 4] of (n, t, h, w)."""
     qx = np.ascontiguousarray(qx, dtype=np.int8)
@@ -144,6 +162,16 @@ def f32_to_bf16(values):
     L = lib()
     return np.array([L.oracle_f32_to_bf16(ctypes.c_float(float(f))) for f in v],
                     dtype=np.uint16).reshape(np.shape(values))
+
+
+def layer_carry(x_ext_bits, w_bits, bias_bits=None):
+    """One streamed chunk: x_ext (bf16 bits [N,T+2,H,W,Cin], the two carried frames
+    first) is quantised as one tensor; the output covers the T chunk frames."""
+    qw, s_w = quantize_weights(w_bits)
+    qx, s_a = act_quant(x_ext_bits)
+    acc = conv_acc_carry(qx, qw)
+    out = epilogue(acc, s_a, s_w, bias_bits)
+    return {"qw": qw, "s_w": s_w, "qx": qx, "s_a": s_a, "acc": acc, "out": out}
 
 
 def layer(x_bits, w_bits, bias_bits=None):

@@ -141,21 +141,25 @@ int oracle_act_quant(const uint16_t *x, int64_t numel, int8_t *qx, float *s_a)
  * zero frames in time, one zero pixel on each spatial side).
  * qx: [N][T][H][W][Cin] (channels_last); qw: [Cout][Cin][3][3][3].
  */
-static int conv_point(const int8_t *qx, const int8_t *qw, int64_t T, int64_t H,
-                      int64_t W, int32_t Cin, int64_t n, int64_t t, int64_t h,
+static int conv_point(const int8_t *qx, const int8_t *qw, int64_t T, int64_t hist,
+                      int64_t H, int64_t W, int32_t Cin, int64_t n, int64_t t, int64_t h,
                       int64_t w, int32_t co, int32_t *out)
 {
+    /* The input holds hist + T frames: hist carried frames, then the T frames
+     * of this call.  Output frame t reads input frames t + kt - 2 + hist for
+     * kt = 0, 1, 2; a frame before the first one is a causal zero frame. */
+    const int64_t Tin = T + hist;
     int64_t acc = 0;
     for (int kt = 0; kt < 3; ++kt) {
-        int64_t ti = t + kt - 2;
-        if (ti < 0 || ti >= T) continue;
+        int64_t ti = t + kt - 2 + hist;
+        if (ti < 0 || ti >= Tin) continue;
         for (int kh = 0; kh < 3; ++kh) {
             int64_t hi = h + kh - 1;
             if (hi < 0 || hi >= H) continue;
             for (int kw = 0; kw < 3; ++kw) {
                 int64_t wi = w + kw - 1;
                 if (wi < 0 || wi >= W) continue;
-                const int8_t *xp = qx + ((((n * T + ti) * H + hi) * W + wi) * Cin);
+                const int8_t *xp = qx + ((((n * Tin + ti) * H + hi) * W + wi) * Cin);
                 for (int32_t ci = 0; ci < Cin; ++ci) {
                     int64_t widx = ((((int64_t)co * Cin + ci) * 3 + kt) * 3 + kh) * 3 + kw;
                     acc += (int64_t)xp[ci] * (int64_t)qw[widx];
@@ -168,9 +172,10 @@ static int conv_point(const int8_t *qx, const int8_t *qw, int64_t T, int64_t H,
     return ORC_OK;
 }
 
-/* Every output point; acc: [N][T][H][W][Cout]. */
-int oracle_conv_acc(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
-                    int64_t H, int64_t W, int32_t Cin, int32_t Cout, int32_t *acc)
+/* Every output point of a call whose input carries `hist` frames of history
+ * (qx: [N][hist + T][H][W][Cin]); acc: [N][T][H][W][Cout]. */
+static int conv_acc_hist(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T, int64_t hist,
+                         int64_t H, int64_t W, int32_t Cin, int32_t Cout, int32_t *acc)
 {
     if (N <= 0 || T <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0) return ORC_ERR_ARG;
     int rc_all = ORC_OK;
@@ -181,7 +186,7 @@ int oracle_conv_acc(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
         for (int64_t w = 0; w < W; ++w)
             for (int32_t co = 0; co < Cout; ++co) {
                 int32_t v = 0;
-                int rc = conv_point(qx, qw, T, H, W, Cin, n, t, h, w, co, &v);
+                int rc = conv_point(qx, qw, T, hist, H, W, Cin, n, t, h, w, co, &v);
                 if (rc != ORC_OK) {
 #pragma omp atomic write
                     rc_all = rc;
@@ -190,6 +195,23 @@ int oracle_conv_acc(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
             }
     }
     return rc_all;
+}
+
+/* Every output point of the causal conv (two zero frames before frame 0);
+ * qx: [N][T][H][W][Cin], acc: [N][T][H][W][Cout]. */
+int oracle_conv_acc(const int8_t *qx, const int8_t *qw, int64_t N, int64_t T,
+                    int64_t H, int64_t W, int32_t Cin, int32_t Cout, int32_t *acc)
+{
+    return conv_acc_hist(qx, qw, N, T, 0, H, W, Cin, Cout, acc);
+}
+
+/* Streaming decode of a chunk of T frames: the two frames before it are the
+ * last two input frames of the previous chunk (carried), not zeros.
+ * qx_ext: [N][T + 2][H][W][Cin] (carried frames first), acc: [N][T][H][W][Cout]. */
+int oracle_conv_acc_carry(const int8_t *qx_ext, const int8_t *qw, int64_t N, int64_t T,
+                          int64_t H, int64_t W, int32_t Cin, int32_t Cout, int32_t *acc)
+{
+    return conv_acc_hist(qx_ext, qw, N, T, 2, H, W, Cin, Cout, acc);
 }
 
 /* Selected output pixels only; pts: [npts][4] = (n, t, h, w); acc: [npts][Cout]. */
@@ -206,7 +228,7 @@ int oracle_conv_acc_points(const int8_t *qx, const int8_t *qw, int64_t N, int64_
         for (int32_t co = 0; co < Cout; ++co) {
             int32_t v = 0;
             int rc = bad ? ORC_ERR_ARG
-                         : conv_point(qx, qw, T, H, W, Cin, q[0], q[1], q[2], q[3], co, &v);
+                         : conv_point(qx, qw, T, 0, H, W, Cin, q[0], q[1], q[2], q[3], co, &v);
             if (rc != ORC_OK) {
 #pragma omp atomic write
                 rc_all = rc;

@@ -347,3 +347,66 @@ def test_layer_close_to_float64_conv_of_bf16_inputs():
     got = b2f(r["out"]).astype(np.float64)
     err = np.abs(got - y).max() / np.abs(y).max()
     assert err < 0.05
+
+
+# ------------------------------------------------- streamed chunks (carried frames)
+
+def _brute_carry(qx_ext, qw):
+    """Pure-Python reference for one streamed chunk: output frame t reads input frames
+    t, t+1, t+2 of the extended input (two carried frames first), spatial padding 1."""
+    N, T2, H, W, Cin = qx_ext.shape
+    Cout = qw.shape[0]
+    out = np.zeros((N, T2 - 2, H, W, Cout), dtype=np.int64)
+    for n in range(N):
+        for t in range(T2 - 2):
+            for h in range(H):
+                for w in range(W):
+                    for co in range(Cout):
+                        s = 0
+                        for kt in range(3):
+                            for kh in range(3):
+                                for kw in range(3):
+                                    hi, wi = h + kh - 1, w + kw - 1
+                                    if 0 <= hi < H and 0 <= wi < W:
+                                        for ci in range(Cin):
+                                            s += int(qx_ext[n, t + kt, hi, wi, ci]) * int(qw[co, ci, kt, kh, kw])
+                        out[n, t, h, w, co] = s
+    return out
+
+
+def test_carry_matches_brute_force_tiny():
+    rng = np.random.default_rng(41)
+    qx_ext = rng.integers(-127, 128, size=(2, 4, 2, 3, 3), dtype=np.int8)   # T = 2 chunk frames
+    qw = rng.integers(-127, 128, size=(2, 3, 3, 3, 3), dtype=np.int8)
+    assert np.array_equal(oracle.conv_acc_carry(qx_ext, qw), _brute_carry(qx_ext, qw))
+
+
+def test_carry_with_zero_history_is_the_causal_conv():
+    rng = np.random.default_rng(42)
+    qx = rng.integers(-127, 128, size=(1, 3, 5, 6, 32), dtype=np.int8)
+    qw = rng.integers(-127, 128, size=(8, 32, 3, 3, 3), dtype=np.int8)
+    ext = np.concatenate([np.zeros_like(qx[:, :2]), qx], axis=1)
+    assert np.array_equal(oracle.conv_acc_carry(ext, qw), oracle.conv_acc(qx, qw))
+
+
+def test_chunked_stream_reproduces_the_whole_sequence():
+    # with the same codes, chunks of two frames that carry the previous chunk's
+    # last two input frames give the whole sequence's accumulators exactly
+    rng = np.random.default_rng(43)
+    qx = rng.integers(-127, 128, size=(2, 7, 4, 5, 32), dtype=np.int8)
+    qw = rng.integers(-127, 128, size=(8, 32, 3, 3, 3), dtype=np.int8)
+    full = oracle.conv_acc(qx, qw)
+    parts = [oracle.conv_acc(qx[:, 0:2], qw)]
+    for t0 in range(2, 7, 2):
+        parts.append(oracle.conv_acc_carry(qx[:, t0 - 2:min(t0 + 2, 7)], qw))
+    assert np.array_equal(np.concatenate(parts, axis=1), full)
+
+
+def test_layer_carry_zero_history_equals_layer():
+    # zero frames leave the absmax, hence the scale and codes, unchanged
+    t = synth.draw_custom(synth.LayerShape(32, 32, 6, 5, T=2), seed=44, outliers=True)
+    xb, wb, bb = (t.x.view(torch.int16).numpy().view(np.uint16), t.w.view(torch.int16).numpy().view(np.uint16),
+                  t.bias.view(torch.int16).numpy().view(np.uint16))
+    ext = np.concatenate([np.zeros_like(xb[:, :2]), xb], axis=1)
+    a, b = oracle.layer_carry(ext, wb, bb), oracle.layer(xb, wb, bb)
+    assert a["s_a"] == b["s_a"] and np.array_equal(a["out"], b["out"])
