@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--layer", type=int, default=0, help="layer index inside the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="decode a multi-frame layer as a stream of chunks of this many frames, each "
+                         "carrying the previous chunk's last two input frames (0: whole layer at once)")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="timed steps as CUDA-graph replays (one graph per buffer set) or direct launches")
     return ap.parse_args()
@@ -275,15 +278,51 @@ def run_ours(args):
             out=torch.empty((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device=dev),
             packed=packed0.clone()))
 
+    # Streamed decode (--chunk C, one video): chunk k covers frames
+    # [kC, kC + C); its input is the view x[:, kC - 2 : kC + C] (the two frames
+    # before it carried), quantised as one tensor, then the carried-frame
+    # convolution; chunk 0 has no history and runs the causal convolution.
+    chunk = args.chunk if (args.chunk > 0 and s.T > args.chunk) else 0
+    if chunk and s.N != 1:
+        raise SystemExit("--chunk streams one video (N = 1)")
+    starts = list(range(0, s.T, chunk)) if chunk else [0]
+    if chunk:
+        for st in sets:
+            st["chunks"] = []
+            for k, t0 in enumerate(starts):
+                t1 = min(t0 + chunk, s.T)
+                xv = st["x"][:, (t0 - 2 if k else 0):t1]
+                st["chunks"].append(dict(
+                    k=k, x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
+                    x_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                    ws=torch.empty(qvae.qvae_act_workspace_bytes(xv.numel()), dtype=torch.uint8, device=dev),
+                    out=st["out"][:, t0:t1]))
+            del st["xq"]
+
+    def act_one(c):
+        qvae.qvae_act_absmax_quant(c["x"], c["xq"], c["x_scale"], c["ws"], stream)
+
+    def conv_one(c, packed):
+        if c.get("k", 0) == 0:
+            qvae.qvae_causal_conv3d_w8a8(c["xq"], c["x_scale"], packed, s_w, b, c["out"], stream)
+        else:
+            qvae.qvae_causal_conv3d_w8a8_carry(c["xq"], c["x_scale"], packed, s_w, b, c["out"], stream)
+
+    def parts(st):
+        return st["chunks"] if chunk else [st]
+
     def act(st):
-        qvae.qvae_act_absmax_quant(st["x"], st["xq"], st["x_scale"], st["ws"], stream)
+        for c in parts(st):
+            act_one(c)
 
     def conv(st):
-        qvae.qvae_causal_conv3d_w8a8(st["xq"], st["x_scale"], st["packed"], s_w, b, st["out"], stream)
+        for c in parts(st):
+            conv_one(c, st["packed"])
 
     def step(st):
-        act(st)
-        conv(st)
+        for c in parts(st):
+            act_one(c)
+            conv_one(c, st["packed"])
 
     # One CUDA graph per buffer set holds that set's step (the three kernels,
     # with their programmatic launch dependencies): a replay costs the host one
@@ -408,7 +447,8 @@ def run_ours(args):
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
                    "launch": ("one CUDA graph replay per step (act absmax, act quantise, conv)"
                               if args.launch == "graph" else "direct launches from Python"),
-                   "ops_per_layer": ops},
+                   "ops_per_layer": ops,
+                   "stream_chunk": (f"{chunk} frames, two carried" if chunk else None)},
         "ms_per_layer": {"step": ms_per_step, "act_absmax_quant": statistics.mean(act_ms),
                          "conv": conv_mean, "conv_median": statistics.median(conv_ms)},
         "conv_tops": conv_tops,
@@ -420,7 +460,7 @@ def run_ours(args):
                      "kernel": "conv3d_w8a8_kernel", "kernel_ms_mean": conv_mean, "launches": R},
         "e2e": {"value": ops * world / (e2e_ms_max * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": s.pixels * s.Cout * 2},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 3 * K * len(starts),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:

@@ -153,6 +153,30 @@ int qvae_causal_conv3d_w8a8(const qvae_shape* shape, const int8_t* xq, const flo
 int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
                                   const int8_t* wq_packed, int32_t* acc, void* stream);
 
+/*
+ * Streamed temporal decode (a video decoded in chunks of frames, as for the
+ * Wan VAE the release note names): the same convolution over a chunk of
+ * shape->T frames whose input carries, in front of the chunk, the last two
+ * input frames of the previous chunk instead of the two causal zero frames:
+ *   acc[n,t,h,w,co] = sum over kt,kh,kw,ci of
+ *                     xq_ext[n, t+kt, h+kh-1, w+kw-1, ci] * wq[co, ci, kt, kh, kw]
+ *   xq_ext     [N][T+2][H][W][Cin] INT8 codes of the extended input, quantised as
+ *              one tensor by qvae_act_absmax_quant (so x_scale covers the carried
+ *              frames too); frames 0 and 1 are the carried ones.
+ *   out_bf16   [N][T][H][W][Cout], the chunk's frames only.
+ * With zero carried frames this equals qvae_causal_conv3d_w8a8 on the chunk;
+ * with the same codes, chunks that carry their predecessors' last two frames
+ * reproduce the whole sequence's accumulators.  Same arguments, layout and
+ * errors as qvae_causal_conv3d_w8a8 otherwise.
+ */
+int qvae_causal_conv3d_w8a8_carry(const qvae_shape* shape, const int8_t* xq_ext, const float* x_scale,
+                                  const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
+                                  void* out_bf16, void* stream);
+
+/* The streamed-chunk convolution writing raw INT32 accumulators [N][T][H][W][Cout]. */
+int qvae_causal_conv3d_w8a8_carry_acc32(const qvae_shape* shape, const int8_t* xq_ext,
+                                        const int8_t* wq_packed, int32_t* acc, void* stream);
+
 /* ---------------------------------------------------------- layer chain -- */
 
 /*

@@ -69,6 +69,7 @@ struct ConvArgs {
   int G;                      // taps per weight stage (1 or 3; 9 / G stages per 128-channel chunk)
   int split;                  // per-sub-tile accumulator hand-off (one accumulator buffer, MS >= 2, SB >= 9 / G)
   int epi_bufs;               // staging buffers per epilogue warp (1 or 2)
+  int carry;                  // 1: the input holds two carried frames before frame 0 (streamed chunk)
   uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
   uint32_t a_box_bytes;       // bytes one activation box delivers
   uint32_t b_tap_bytes;       // weight rows this CTA loads per tap x 128 B
@@ -175,7 +176,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   };
   for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
     const TileCoord c = decode_tile<kPair>(a, tile, rank);
-    const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
+    const int kt_lo = (a.carry || c.t >= 2) ? 0 : 2 - c.t;  // taps that meet causal zero frames are skipped
     const int nkb = (3 - kt_lo) * a.nchunks;
     const uint32_t d_tile = r.tmem_base + cs * static_cast<uint32_t>(kMS) * nt;
     const uint32_t accb = cs * static_cast<uint32_t>(kMS);  // this buffer's first barrier index
@@ -381,10 +382,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     bool waited = false;
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
-      const int kt_lo = c.t >= 2 ? 0 : 2 - c.t;
+      const int kt_lo = (a.carry || c.t >= 2) ? 0 : 2 - c.t;
       const int nkb = (3 - kt_lo) * a.nchunks;
       for (int kb = 0; kb < nkb; ++kb) {
         const int kt = kt_lo + kb / a.nchunks, ch = kb % a.nchunks;
+        const int frame = c.t + kt - 2 + 2 * a.carry;  // input frame of temporal tap kt
         if (!waited) {
           for (; preissued < a.SB && preissued < ngrp; ++preissued)
             if (!load_b(c, kt, ch, preissued)) goto producer_done;
@@ -397,10 +399,10 @@ __global__ void __launch_bounds__(kConvThreads, 1)
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
           if (kPair) {
             tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * 128, c.w0 - 1,
-                             c.h0 - 1, c.t + kt - 2, c.n);
+                             c.h0 - 1, frame, c.n);
           } else {
-            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1,
-                        c.t + kt - 2, c.n);
+            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1, frame,
+                        c.n);
           }
         }
         a_armed |= 1u << as;

@@ -280,11 +280,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// carry: xq holds T + 2 frames per batch item, the first two carried from
+// the previous chunk of a streamed video (output frames are the last T).
 int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                 const int8_t* wq, const float* w_scale, const void* bias, void* out, int32_t* acc,
-                cudaStream_t stream) {
+                cudaStream_t stream, bool carry = false) {
   int rc = check_shape(shape);
   if (rc) return rc;
+  if (carry && (static_cast<double>(shape->T + 2) * shape->H * shape->W * shape->Cin >= 1099511627776.0))
+    return QVAE_ERR_SHAPE;
   const bool acc_mode = acc != nullptr;
   const qvae_shape& s = *shape;
   if (pixels(s) == 0) return QVAE_OK;  // nothing to read or write
@@ -303,13 +307,13 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
 
   CUtensorMap tmap_x, tmap_w, tmap_out;
   {
+    const cuuint64_t t_in = static_cast<cuuint64_t>(s.T) + (carry ? 2 : 0);
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W),
-                                static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.T),
-                                static_cast<cuuint64_t>(s.N)};
+                                static_cast<cuuint64_t>(s.H), t_in, static_cast<cuuint64_t>(s.N)};
     const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin),
                                    static_cast<cuuint64_t>(s.W) * s.Cin,
                                    static_cast<cuuint64_t>(s.H) * s.W * s.Cin,
-                                   static_cast<cuuint64_t>(s.T) * s.H * s.W * s.Cin};
+                                   t_in * s.H * s.W * s.Cin};
     const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(qvae::kBoxW),
                                static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
     rc = encode_map(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims, strides, box, 5,
@@ -366,6 +370,7 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.G = t.G;
   a.split = t.split ? 1 : 0;
   a.epi_bufs = t.epi_bufs;
+  a.carry = carry ? 1 : 0;
   a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
@@ -631,6 +636,20 @@ int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
   if (!acc) return QVAE_ERR_ARG;
   return launch_conv(shape, xq, nullptr, wq_packed, nullptr, nullptr, nullptr, acc,
                      static_cast<cudaStream_t>(stream));
+}
+
+int qvae_causal_conv3d_w8a8_carry(const qvae_shape* shape, const int8_t* xq_ext, const float* x_scale,
+                                  const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
+                                  void* out_bf16, void* stream) {
+  return launch_conv(shape, xq_ext, x_scale, wq_packed, w_scale, bias_bf16, out_bf16, nullptr,
+                     static_cast<cudaStream_t>(stream), true);
+}
+
+int qvae_causal_conv3d_w8a8_carry_acc32(const qvae_shape* shape, const int8_t* xq_ext,
+                                        const int8_t* wq_packed, int32_t* acc, void* stream) {
+  if (!acc) return QVAE_ERR_ARG;
+  return launch_conv(shape, xq_ext, nullptr, wq_packed, nullptr, nullptr, nullptr, acc,
+                     static_cast<cudaStream_t>(stream), true);
 }
 
 int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,

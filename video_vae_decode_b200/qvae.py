@@ -28,6 +28,7 @@ EXPORTS = (
     "qvae_decode_layers", "qvae_get_error", "qvae_set_wait_limit_ns",
     "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
     "qvae_act_absmax_quant_noalloc", "qvae_set_act_passes",
+    "qvae_causal_conv3d_w8a8_carry", "qvae_causal_conv3d_w8a8_carry_acc32",
 )
 
 
@@ -70,6 +71,8 @@ def lib():
             "qvae_act_absmax_quant_noalloc": ([p, i64, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_carry": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_carry_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
             "qvae_decode_layers": ([ctypes.POINTER(qvae_layer), i32, p, sz, p], ctypes.c_int),
             "qvae_get_error": ([p], ctypes.c_int),
@@ -194,6 +197,47 @@ def causal_conv3d_w8a8(xq, x_scale, wq_packed, w_scale, bias, Cout: int, stream=
     out = torch.empty(tuple(xq.shape[:-1]) + (Cout,), dtype=torch.bfloat16, device=xq.device)
     qvae_causal_conv3d_w8a8(xq, x_scale, wq_packed, w_scale, bias, out, stream)
     return out
+
+
+def _chunk_shape(xq_ext: torch.Tensor, Cout: int) -> qvae_shape:
+    """Shape of a streamed chunk: xq_ext holds two carried frames before the chunk's."""
+    N, T2, H, W, Cin = xq_ext.shape
+    if T2 < 2:
+        raise ValueError("a streamed chunk's input holds two carried frames before its own")
+    return make_shape(N, T2 - 2, H, W, Cin, Cout)
+
+
+def qvae_causal_conv3d_w8a8_carry(xq_ext: torch.Tensor, x_scale: torch.Tensor, wq_packed: torch.Tensor,
+                                  w_scale: torch.Tensor, bias: Optional[torch.Tensor], out: torch.Tensor,
+                                  stream=None) -> None:
+    shp = _chunk_shape(xq_ext, int(out.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_carry",
+           lib().qvae_causal_conv3d_w8a8_carry(ctypes.byref(shp), _ptr(xq_ext), _ptr(x_scale), _ptr(wq_packed),
+                                               _ptr(w_scale), _ptr(bias), _ptr(out), _stream(stream)))
+
+
+def qvae_causal_conv3d_w8a8_carry_acc32(xq_ext: torch.Tensor, wq_packed: torch.Tensor, acc: torch.Tensor,
+                                        stream=None) -> None:
+    shp = _chunk_shape(xq_ext, int(acc.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_carry_acc32",
+           lib().qvae_causal_conv3d_w8a8_carry_acc32(ctypes.byref(shp), _ptr(xq_ext), _ptr(wq_packed),
+                                                     _ptr(acc), _stream(stream)))
+
+
+def conv_carry(xq_ext, x_scale, wq_packed, w_scale, bias, Cout: int, stream=None):
+    _chunk_shape(xq_ext, Cout)
+    N, T2, H, W, _ = xq_ext.shape
+    out = torch.empty((N, T2 - 2, H, W, Cout), dtype=torch.bfloat16, device=xq_ext.device)
+    qvae_causal_conv3d_w8a8_carry(xq_ext, x_scale, wq_packed, w_scale, bias, out, stream)
+    return out
+
+
+def conv_carry_acc32(xq_ext, wq_packed, Cout: int, stream=None):
+    _chunk_shape(xq_ext, Cout)
+    N, T2, H, W, _ = xq_ext.shape
+    acc = torch.empty((N, T2 - 2, H, W, Cout), dtype=torch.int32, device=xq_ext.device)
+    qvae_causal_conv3d_w8a8_carry_acc32(xq_ext, wq_packed, acc, stream)
+    return acc
 
 
 def conv_acc32(xq, wq_packed, Cout: int, stream=None):
