@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--chunk", type=int, default=0,
                     help="decode a multi-frame layer as a stream of chunks of this many frames, each "
                          "carrying the previous chunk's last two input frames (0: whole layer at once)")
+    ap.add_argument("--chain", default="",
+                    help="comma-separated consecutive layers of the workload run as one qvae_decode_layers "
+                         "chain, each output feeding the next input (one GPU)")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="timed steps as CUDA-graph replays (one graph per buffer set) or direct launches")
     return ap.parse_args()
@@ -471,10 +474,102 @@ def run_ours(args):
     return 0
 
 
+def run_chain(args):
+    """Layers of a workload as one qvae_decode_layers chain on one GPU.
+
+    Each layer's output buffer is the next layer's input, so the library takes
+    each input's absmax from the previous convolution's epilogue and runs only
+    the quantise pass.  The same layers with separate input buffers (no
+    chaining) are timed too, as `unchained_ms_per_step`.
+    """
+    import math
+    import torch
+    from video_vae_decode_b200 import qvae, synth
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    idx = [int(v) for v in args.chain.split(",")]
+    wl = synth.WORKLOADS[args.workload]
+    tens = synth.draw_workload(args.workload, seed=wl.seed, only=idx)
+    for a, b in zip(tens, tens[1:]):
+        sa, sb = a.shape, b.shape
+        if (sa.N, sa.T, sa.H, sa.W, sa.Cout) != (sb.N, sb.T, sb.H, sb.W, sb.Cin):
+            raise SystemExit(f"layers {idx} do not chain: {sa} -> {sb}")
+    weights = []
+    for t in tens:
+        packed, s_w = qvae.quantize_weights(t.w.to(dev))
+        weights.append((packed, s_w, t.bias.to(dev)))
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    per_set = sum(t.x.numel() * 2 + t.shape.pixels * t.shape.Cout * 2 for t in tens)
+    n_sets = max(2, math.ceil(3 * L2_BYTES / per_set))
+
+    def make_set(chained):
+        x0 = tens[0].x.to(dev)
+        specs, x = [], x0
+        for k, t in enumerate(tens):
+            if k and not chained:
+                x = torch.empty_like(x)  # a separate input buffer: no chaining
+            out = torch.empty((t.shape.N, t.shape.T, t.shape.H, t.shape.W, t.shape.Cout),
+                              dtype=torch.bfloat16, device=dev)
+            packed, s_w, b = weights[k]
+            specs.append(dict(x=x, out=out, wq_packed=packed.clone(), w_scale=s_w, bias=b, quantized=True))
+            x = out
+        layers = qvae.make_layers(specs)
+        ws = torch.empty(qvae.qvae_decode_workspace_bytes(layers), dtype=torch.uint8, device=dev)
+        return dict(specs=specs, layers=layers, ws=ws)
+
+    def timed(chained):
+        sets = [make_set(chained) for _ in range(n_sets)]
+        graphs = []
+        qvae.qvae_decode_layers(sets[0]["layers"], sets[0]["ws"], stream)
+        torch.cuda.synchronize()
+        for st in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                qvae.qvae_decode_layers(st["layers"], st["ws"], stream)
+            graphs.append(g)
+        for i in range(args.warmup):
+            graphs[i % n_sets].replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(0) as clk:
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[i % n_sets].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        if qvae.qvae_get_error() != 0:
+            raise RuntimeError("device-side timeout")
+        del graphs, sets
+        return e0.elapsed_time(e1) / args.steps, clk.summary()
+
+    ms, clocks = timed(True)
+    ms_unchained, _ = timed(False)
+    ops = sum(t.shape.ops() for t in tens)
+    line = {
+        "metric": METRIC + ", layer chain", "value": ops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, f32 epilogue, bf16 io",
+        "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
+        "config": {"workload": args.workload, "chain": [layer_name(t) for t in tens],
+                   "l2": f"{n_sets} buffer sets rotate ({n_sets * per_set / 2**20:.0f} MiB)",
+                   "launch": "one CUDA graph replay per chain (qvae_decode_layers)", "ops": ops},
+        "unchained_ms_per_step": ms_unchained,
+        "gpu_launches": 3 * len(tens) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.chain:
+        return run_chain(args)
     return run_ours(args)
 
 

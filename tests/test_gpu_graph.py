@@ -1,10 +1,12 @@
-"""The per-layer path (act quantiser + conv, and qvae_decode_layers) inside a CUDA graph.
+"""The per-layer path (act quantiser + conv) and qvae_decode_layers: CUDA-graph replay and
+layer chains.
 
 The library's calls launch on the caller's stream, allocate nothing and never
 synchronise, so a decoder can capture them once and replay.  A replay must
 give bit-identical results to direct calls on the same data, including data
 written into the captured input buffers after the capture.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -95,3 +97,60 @@ def test_decode_layers_replays_in_a_cuda_graph(q):
     assert q.qvae_get_error() == 0
     for sp, ref in zip(specs, refs):
         assert torch.equal(bits(sp["out"]), bits(ref))
+
+
+def _chain(q, shapes, passthrough=(), seed=31):
+    """Layers whose outputs feed the next layer's input (same buffer)."""
+    gen = torch.Generator().manual_seed(seed)
+    t0 = synth.draw_layer(gen, shapes[0], outliers=True)
+    x = t0.x.cuda()
+    specs, weights = [], []
+    for i, s in enumerate(shapes):
+        t = t0 if i == 0 else synth.draw_layer(gen, s, outliers=False)
+        w, b = t.w.cuda(), t.bias.cuda()
+        packed, s_w = q.quantize_weights(w)
+        out = torch.zeros((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
+        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=i not in passthrough))
+        weights.append((packed, s_w, b, s.Cout))
+        x = out
+    return specs, weights
+
+
+def _layer_by_layer(q, specs, weights):
+    """Reference: each layer on its actual input with the standalone absmax pass."""
+    outs = []
+    for sp, (packed, s_w, b, Cout) in zip(specs, weights):
+        if not sp["quantized"]:
+            outs.append(sp["out"].clone())
+            continue
+        xq, s_a = q.act_absmax_quant(sp["x"])
+        outs.append(q.causal_conv3d_w8a8(xq, s_a, packed, s_w, b, Cout))
+    return outs
+
+
+@pytest.mark.parametrize("passthrough", [(), (1,)])
+def test_decode_chain_takes_each_input_absmax_from_the_previous_epilogue(q, passthrough):
+    # ragged sizes: the epilogue's maximum must skip rows and columns beyond the image
+    shapes = [synth.LayerShape(96, 192, 37, 21, T=2), synth.LayerShape(192, 192, 37, 21, T=2),
+              synth.LayerShape(192, 96, 37, 21, T=2)]
+    specs, weights = _chain(q, shapes, passthrough)
+    layers = q.make_layers(specs)
+    ws = torch.empty(q.qvae_decode_workspace_bytes(layers), dtype=torch.uint8, device="cuda")
+    q.qvae_decode_layers(layers, ws)
+    torch.cuda.synchronize()
+    assert q.qvae_get_error() == 0
+    got = [sp["out"].clone() for sp in specs]
+    want = _layer_by_layer(q, specs, weights)
+    for g, w_ in zip(got, want):
+        assert torch.equal(g.view(torch.int16), w_.view(torch.int16))
+    # and the first layer against the oracle
+    ref = oracle_layer(specs[0], q)
+    assert np.array_equal(got[0].cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+def oracle_layer(sp, q):
+    import oracle
+    gen = torch.Generator().manual_seed(31)
+    t = synth.draw_layer(gen, synth.LayerShape(96, 192, 37, 21, T=2), outliers=True)
+    b = lambda v: v.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return oracle.layer(b(t.x), b(t.w), b(t.bias))["out"]

@@ -79,6 +79,7 @@ struct ConvArgs {
   const float* w_scale;       // [Cout]
   const __nv_bfloat16* bias;  // [Cout] or null
   int32_t* acc_out;           // [N,T,H,W,Cout] (accumulator mode)
+  uint32_t* out_amax;         // or null: max |bf16 output| (15-bit magnitude) accumulated here
   uint64_t wait_limit_ns;
 };
 
@@ -487,6 +488,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     const uint32_t empty_leader = kPair ? map_to_cta(acc_empty, 0) : acc_empty;
     uint32_t cs = 0, cp = 0;
     int scale_co0 = -1;
+    uint32_t out_max = 0;  // largest |output| written by this lane (bf16 magnitude bits)
     bool dead = false;  // a wait gave up: keep pace with the other warps' table barriers, do no work
     // Scale and bias table for output channels co0..co0+NT-1.  Every epilogue
     // warp sees the same tiles, so all of them take part; the first barrier
@@ -551,6 +553,15 @@ __global__ void __launch_bounds__(kConvThreads, 1)
               packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
               packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
             }
+            if (a.out_amax) {
+              // the next layer's activation absmax, taken on what is written
+              const int h = c.h0 + s * kTileRows + row / kTileW;
+              const int w = c.w0 + row % kTileW;
+              if (h < a.H && w < a.W) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) out_max = max(out_max, max(packed[e] & 0x7FFFu, (packed[e] >> 16) & 0x7FFFu));
+              }
+            }
             // the store issued epi_bufs slices ago read this buffer: let it finish
             if (lane == 0) {
               if (a.epi_bufs == 2) {
@@ -607,6 +618,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
     }
     if (!kAcc32 && lane == 0) bulk_wait_group<0>();
+    if (!kAcc32 && a.out_amax) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) out_max = max(out_max, __shfl_xor_sync(0xFFFFFFFFu, out_max, o));
+      if (lane == 0) atomicMax(a.out_amax, out_max);
+    }
   }
 
   // Reconverge every warp (one lane of warps 0 and 1 ran a role alone) before

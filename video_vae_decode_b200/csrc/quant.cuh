@@ -136,7 +136,8 @@ __device__ __forceinline__ uint4 quant16(const Quantizer& z, bool zero, const ui
   return make_uint4(quant4(z, a.x, a.y), quant4(z, a.z, a.w), quant4(z, b.x, b.y), quant4(z, b.z, b.w));
 }
 
-// Pass 2: reduce the partial maxima, derive the scale, write INT8 codes.
+// Pass 2: reduce the partial maxima (or read the one maximum the previous
+// layer's convolution accumulated), derive the scale, write INT8 codes.
 // Group g (g < nvec2 = numel / 16) is 16 values: two 16-byte bf16 vectors in,
 // one 16-byte code vector out.  Groups are visited from the end of the tensor
 // to its start: the re-read of x begins with what pass 1 read last (still in
@@ -146,9 +147,11 @@ __device__ __forceinline__ uint4 quant16(const Quantizer& z, bool zero, const ui
 __global__ void __launch_bounds__(kActThreads) act_quant_kernel(
     const uint4* __restrict__ x, int64_t nvec2, const uint16_t* __restrict__ xs, int64_t numel,
     const uint32_t* __restrict__ partial, int npartial, uint4* __restrict__ xq,
-    int8_t* __restrict__ xq_bytes, float* __restrict__ x_scale) {
+    int8_t* __restrict__ xq_bytes, float* __restrict__ x_scale, uint32_t* zero_word) {
   __shared__ uint32_t red[kActThreads / 32];
   grid_dependents_launch();  // the convolution may start its prologue
+  // a word the following convolution accumulates a maximum into starts at zero
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
   int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;
   const int64_t last = nvec2 - 1;

@@ -11,7 +11,6 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
-#include <mutex>
 #include <string>
 #include <utility>
 
@@ -38,9 +37,7 @@ int g_max_clusters[kMaxDevices] = {0};
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
 
 int cuda_fail(cudaError_t e, const char* what) {
-  char buf[256];
-  std::snprintf(buf, sizeof buf, "%s: %s", what, cudaGetErrorString(e));
-  t_last_error = buf;
+  t_last_error = std::string(what) + ": " + cudaGetErrorString(e);
   return QVAE_ERR_CUDA;
 }
 
@@ -284,7 +281,7 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
 // the previous chunk of a streamed video (output frames are the last T).
 int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                 const int8_t* wq, const float* w_scale, const void* bias, void* out, int32_t* acc,
-                cudaStream_t stream, bool carry = false) {
+                cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr) {
   int rc = check_shape(shape);
   if (rc) return rc;
   if (carry && (static_cast<double>(shape->T + 2) * shape->H * shape->W * shape->Cin >= 1099511627776.0))
@@ -371,6 +368,7 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.split = t.split ? 1 : 0;
   a.epi_bufs = t.epi_bufs;
   a.carry = carry ? 1 : 0;
+  a.out_amax = acc_mode ? nullptr : out_amax;
   a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
   a.tmem_cols = t.tmem_cols;
@@ -505,8 +503,10 @@ bool try_fused_act(int dev, int sms, const void* x, int64_t numel, int8_t* xq, f
   return false;
 }
 
+// zero_word (nullable): a device word the quantise pass sets to zero, for a
+// following convolution to accumulate its output maximum into.
 int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* ws,
-               size_t ws_bytes, cudaStream_t stream) {
+               size_t ws_bytes, cudaStream_t stream, uint32_t* zero_word = nullptr) {
   if (numel < 0) return QVAE_ERR_ARG;
   if (!x_scale) return QVAE_ERR_ARG;
   if (numel == 0) {
@@ -522,7 +522,8 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   // The single pass reads x once but needs a counter reset and a cooperative
   // launch; measured slower than two passes on the decoder top-stage layer
   // (6.3 M values), so it runs only when asked for.
-  if (g_act_mode == 1 && try_fused_act(dev, sms, x, numel, xq, x_scale, ws, ws_bytes, stream, &rc)) return rc;
+  if (g_act_mode == 1 && !zero_word && try_fused_act(dev, sms, x, numel, xq, x_scale, ws, ws_bytes, stream, &rc))
+    return rc;
   const int g1 = act_grid(numel, sms);
   uint32_t* partial = static_cast<uint32_t*>(ws);
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, stream>>>(
@@ -533,7 +534,29 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, stream, 1,
                              static_cast<const uint4*>(x), nvec2, static_cast<const uint16_t*>(x), numel,
                              static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
-                             x_scale));
+                             x_scale, zero_word));
+  return QVAE_OK;
+}
+
+// The quantise pass alone, for an input whose absmax (15-bit bf16 magnitude)
+// the previous convolution accumulated into *amax while writing it.  A plain
+// launch: the input is that convolution's output, so nothing of this kernel
+// may run before it has finished.
+int launch_quant_from_amax(const void* x, int64_t numel, const uint32_t* amax, int8_t* xq, float* x_scale,
+                           uint32_t* zero_word, cudaStream_t stream) {
+  if (numel == 0) {
+    QVAE_CUDA(cudaMemsetAsync(x_scale, 0, sizeof(float), stream));
+    return QVAE_OK;
+  }
+  int dev, sms, rc;
+  if ((rc = current_device(&dev))) return rc;
+  if ((rc = sm_count(dev, &sms))) return rc;
+  const int64_t nvec2 = numel / 16;
+  const int g2 = quant_grid(numel, sms);
+  qvae::act_quant_kernel<<<g2, qvae::kActThreads, 0, stream>>>(
+      static_cast<const uint4*>(x), nvec2, static_cast<const uint16_t*>(x), numel, amax, 1,
+      reinterpret_cast<uint4*>(xq), xq, x_scale, zero_word);
+  QVAE_CUDA(cudaGetLastError());
   return QVAE_OK;
 }
 
@@ -686,7 +709,7 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
   QVAE_CUDA(launch_dependent(qvae::act_quant_kernel, g2, qvae::kActThreads, 0, st, 1,
                              static_cast<const uint4*>(x_bf16), nvec2, static_cast<const uint16_t*>(x_bf16),
                              numel, static_cast<const uint32_t*>(partial), g1, reinterpret_cast<uint4*>(xq), xq,
-                             x_scale));
+                             x_scale, static_cast<uint32_t*>(nullptr)));
   return QVAE_OK;
 }
 
@@ -697,6 +720,15 @@ size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {
     if (layers[i].quantized)
       max_in = std::max<int64_t>(max_in, pixels(layers[i].shape) * layers[i].shape.Cin);
   return align_up(static_cast<size_t>(max_in), 256) + 256 + kActWorkspace;
+}
+
+// Layer i's output is, element for element, layer i + 1's input (both
+// quantised, same pixels, Cout == next Cin, same pointer).
+bool feeds_next(const qvae_layer* layers, int32_t n, int32_t i) {
+  if (i + 1 >= n) return false;
+  const qvae_layer &a = layers[i], &b = layers[i + 1];
+  return a.quantized && b.quantized && a.out == b.x && a.shape.N == b.shape.N && a.shape.T == b.shape.T &&
+         a.shape.H == b.shape.H && a.shape.W == b.shape.W && a.shape.Cout == b.shape.Cin;
 }
 
 int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
@@ -719,15 +751,24 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
   const size_t xq_bytes = need - 256 - kActWorkspace;
   int8_t* xq = reinterpret_cast<int8_t*>(ws);
   float* x_scale = reinterpret_cast<float*>(ws + xq_bytes);
+  // two words of the 256-byte gap: the absmax of layer i's input, accumulated
+  // by layer i - 1's convolution when it writes that input (alternating)
+  uint32_t* amax_word[2] = {reinterpret_cast<uint32_t*>(ws + xq_bytes + 64),
+                            reinterpret_cast<uint32_t*>(ws + xq_bytes + 128)};
   void* partial = ws + xq_bytes + 256;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int32_t i = 0; i < n; ++i) {
     const qvae_layer& L = layers[i];
     if (!L.quantized) continue;
     const int64_t numel = pixels(L.shape) * L.shape.Cin;
-    int rc = launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st);
+    const bool fed = i > 0 && feeds_next(layers, n, i - 1);  // input absmax already accumulated
+    const bool feeds = feeds_next(layers, n, i);            // accumulate the next input's absmax
+    uint32_t* next_amax = feeds ? amax_word[(i + 1) & 1] : nullptr;
+    int rc = fed ? launch_quant_from_amax(L.x, numel, amax_word[i & 1], xq, x_scale, next_amax, st)
+                 : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, next_amax);
     if (rc) return rc;
-    rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st);
+    rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
+                     next_amax);
     if (rc) return rc;
   }
   return QVAE_OK;
