@@ -201,7 +201,11 @@ size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
 /*
  * For each layer with quantized != 0, in order on one stream: activation
  * absmax + quantise into the workspace, then the convolution into `out`.
- * All layers are validated before anything is launched.
+ * All layers are validated before anything is launched.  When a quantised
+ * layer's `out` is the next quantised layer's `x` (same N, T, H, W and
+ * Cout == next Cin), the convolution also accumulates the maximum bf16
+ * magnitude it writes into the workspace and the next layer skips its absmax
+ * pass: codes, scales and outputs are the same as layer-by-layer calls.
  */
 int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
                        size_t workspace_bytes, void* stream);
