@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--chunk", type=int, default=0,
                     help="decode a multi-frame layer as a stream of chunks of this many frames, each "
                          "carrying the previous chunk's last two input frames (0: whole layer at once)")
+    ap.add_argument("--bands", type=int, default=0,
+                    help="decode one image layer in this many row bands (tiled decode: whole-image "
+                         "absmax, then per band quantise + band convolution)")
     ap.add_argument("--chain", default="",
                     help="comma-separated consecutive layers of the workload run as one qvae_decode_layers "
                          "chain, each output feeding the next input (one GPU)")
@@ -302,8 +305,37 @@ def run_ours(args):
                     out=st["out"][:, t0:t1]))
             del st["xq"]
 
+    # Tiled decode (--bands B, one image): the whole image's absmax into a
+    # word, then per band its rows plus halo rows quantised from that word and
+    # the band convolution into the band's output rows.
+    nb = args.bands if args.bands > 1 else 0
+    if nb and s.N * s.T != 1:
+        raise SystemExit("--bands decodes one image (N = T = 1)")
+    if nb and chunk:
+        raise SystemExit("--bands and --chunk do not combine")
+    if nb:
+        from video_vae_decode_b200 import bands as bandlib
+        for st in sets:
+            st["amax"] = torch.empty(1, dtype=torch.int32, device=dev)
+            st["bands"] = []
+            for k in range(nb):
+                r0, r1 = bandlib.band_rows(s.H, nb, k)
+                lo, hi, ht, hb = bandlib.band_input(s.H, r0, r1)
+                xv = st["x"][:, :, lo:hi]
+                st["bands"].append(dict(x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
+                                        x_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                                        ht=ht, hb=hb, out=st["out"][:, :, r0:r1]))
+            del st["xq"]
+
     def act_one(c):
         qvae.qvae_act_absmax_quant(c["x"], c["xq"], c["x_scale"], c["ws"], stream)
+
+    def band_quant(st, c):
+        qvae.qvae_act_quant_from_absmax(c["x"], st["amax"], c["xq"], c["x_scale"], stream)
+
+    def band_conv(st, c):
+        qvae.qvae_causal_conv3d_w8a8_band(c["xq"], c["ht"], c["hb"], c["x_scale"], st["packed"], s_w, b,
+                                          c["out"], stream)
 
     def conv_one(c, packed):
         if c.get("k", 0) == 0:
@@ -315,14 +347,29 @@ def run_ours(args):
         return st["chunks"] if chunk else [st]
 
     def act(st):
+        if nb:
+            qvae.qvae_act_absmax(st["x"], st["amax"], stream)
+            for c in st["bands"]:
+                band_quant(st, c)
+            return
         for c in parts(st):
             act_one(c)
 
     def conv(st):
+        if nb:
+            for c in st["bands"]:
+                band_conv(st, c)
+            return
         for c in parts(st):
             conv_one(c, st["packed"])
 
     def step(st):
+        if nb:
+            qvae.qvae_act_absmax(st["x"], st["amax"], stream)
+            for c in st["bands"]:
+                band_quant(st, c)
+                band_conv(st, c)
+            return
         for c in parts(st):
             act_one(c)
             conv_one(c, st["packed"])
@@ -451,7 +498,8 @@ def run_ours(args):
                    "launch": ("one CUDA graph replay per step (act absmax, act quantise, conv)"
                               if args.launch == "graph" else "direct launches from Python"),
                    "ops_per_layer": ops,
-                   "stream_chunk": (f"{chunk} frames, two carried" if chunk else None)},
+                   "stream_chunk": (f"{chunk} frames, two carried" if chunk else None),
+                   "row_bands": nb or None},
         "ms_per_layer": {"step": ms_per_step, "act_absmax_quant": statistics.mean(act_ms),
                          "conv": conv_mean, "conv_median": statistics.median(conv_ms)},
         "conv_tops": conv_tops,
@@ -463,7 +511,7 @@ def run_ours(args):
                      "kernel": "conv3d_w8a8_kernel", "kernel_ms_mean": conv_mean, "launches": R},
         "e2e": {"value": ops * world / (e2e_ms_max * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": s.pixels * s.Cout * 2},
-        "gpu_launches": 3 * K * len(starts),
+        "gpu_launches": K * (1 + 2 * nb if nb else 3 * len(starts)),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:

@@ -128,6 +128,25 @@ int qvae_act_absmax_quant(const void* x_bf16, int64_t numel, int8_t* xq, float* 
 int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
                                   void* stream);
 
+/*
+ * The two activation steps apart, for a scale taken over more than the
+ * tensor at hand (the row bands of one image, on one GPU or several):
+ *   qvae_act_absmax        *amax = max |x| over numel bf16 values, as the
+ *                          15-bit magnitude of a bf16 (an unsigned maximum of
+ *                          such words is the maximum of the values, so the
+ *                          words of several bands or GPUs combine with a
+ *                          plain unsigned max, e.g. an all-reduce MAX);
+ *                          amax is a device uint32, zeroed by the call.
+ *   qvae_act_quant_from_absmax   codes and scale of x for that maximum:
+ *                          scale = bf16(amax) / 127, codes as in
+ *                          qvae_act_absmax_quant.  With *amax from the whole
+ *                          tensor the result equals qvae_act_absmax_quant's.
+ * No workspace.  Errors as qvae_act_absmax_quant.
+ */
+int qvae_act_absmax(const void* x_bf16, int64_t numel, uint32_t* amax, void* stream);
+int qvae_act_quant_from_absmax(const void* x_bf16, int64_t numel, const uint32_t* amax, int8_t* xq,
+                               float* x_scale, void* stream);
+
 /* ---------------------------------------------------------- convolution -- */
 
 /*
@@ -176,6 +195,31 @@ int qvae_causal_conv3d_w8a8_carry(const qvae_shape* shape, const int8_t* xq_ext,
 /* The streamed-chunk convolution writing raw INT32 accumulators [N][T][H][W][Cout]. */
 int qvae_causal_conv3d_w8a8_carry_acc32(const qvae_shape* shape, const int8_t* xq_ext,
                                         const int8_t* wq_packed, int32_t* acc, void* stream);
+
+/*
+ * Row-band decode (tiled decode for memory, which the dsh-qwen-paint plugin
+ * README falls back to when a VAE decode runs out of memory; and the split of
+ * one image across GPUs): the convolution of output rows [r0, r0 + shape->H),
+ * of an image, from an input band holding those rows plus halo_top (0 or 1) rows above
+ * and halo_bot (0 or 1) rows below:
+ *   xq_band  [N][T][halo_top + H + halo_bot][W][Cin] codes, quantised with the
+ *            scale of the whole image (qvae_act_absmax over every band, then
+ *            qvae_act_quant_from_absmax per band);
+ *   out_bf16 [N][T][H][W][Cout], the band's output rows.
+ * A missing halo (0) is the image edge: zero padding.  Output row h reads
+ * input rows h + halo_top - 1 .. h + halo_top + 1.  Bands that tile the
+ * image, each with the neighbouring rows as halos, give exactly the
+ * whole-image convolution.  Errors as qvae_causal_conv3d_w8a8;
+ * QVAE_ERR_ARG for a halo outside 0..1.
+ */
+int qvae_causal_conv3d_w8a8_band(const qvae_shape* shape, int32_t halo_top, int32_t halo_bot,
+                                 const int8_t* xq_band, const float* x_scale, const int8_t* wq_packed,
+                                 const float* w_scale, const void* bias_bf16, void* out_bf16, void* stream);
+
+/* The row-band convolution writing raw INT32 accumulators [N][T][H][W][Cout]. */
+int qvae_causal_conv3d_w8a8_band_acc32(const qvae_shape* shape, int32_t halo_top, int32_t halo_bot,
+                                       const int8_t* xq_band, const int8_t* wq_packed, int32_t* acc,
+                                       void* stream);
 
 /* ---------------------------------------------------------- layer chain -- */
 

@@ -35,6 +35,8 @@ def lib():
         L.oracle_act_absmax.argtypes = [p, i64, p]
         L.oracle_act_absmax.restype = ctypes.c_int
         L.oracle_act_quant.argtypes = [p, i64, p, p]
+        L.oracle_act_quant_amax.argtypes = [p, i64, f32, p, p]
+        L.oracle_act_quant_amax.restype = ctypes.c_int
         L.oracle_act_quant.restype = ctypes.c_int
         L.oracle_conv_acc.argtypes = [p, p, i64, i64, i64, i64, i32, i32, p]
         L.oracle_conv_acc.restype = ctypes.c_int
@@ -99,6 +101,15 @@ def act_quant(x_bits):
     qx = np.empty(x.shape, dtype=np.int8)
     s = np.zeros(1, dtype=np.float32)
     _check(lib().oracle_act_quant(_ptr(x), x.size, _ptr(qx), _ptr(s)), "act_quant")
+    return qx, s[0]
+
+
+def act_quant_amax(x_bits, amax):
+    """Codes and scale of x for a maximum |value| taken over a larger tensor."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    qx = np.empty(x.shape, dtype=np.int8)
+    s = np.zeros(1, dtype=np.float32)
+    _check(lib().oracle_act_quant_amax(_ptr(x), x.size, float(amax), _ptr(qx), _ptr(s)), "act_quant_amax")
     return qx, s[0]
 
 

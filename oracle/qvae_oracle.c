@@ -118,18 +118,29 @@ int oracle_act_absmax(const uint16_t *x, int64_t numel, float *amax_out)
 /*
  * Dynamic per-tensor activation quantisation.
  * x: bf16 bits, numel elements.  qx: INT8 codes, same order.  s_a: scale.
+ * oracle_act_quant_amax takes the maximum |x| from the caller: the maximum
+ * over a larger tensor of which x is a part (the row bands of one image);
+ * the codes of every part then equal those of the whole tensor.
  */
+int oracle_act_quant_amax(const uint16_t *x, int64_t numel, float amax, int8_t *qx, float *s_a)
+{
+    amax = amax * 1.0f;              /* activation clip ratio 1.0 */
+    float s = amax / 127.0f;
+    *s_a = s;
+    for (int64_t i = 0; i < numel; ++i) {
+        float v = bf16_bits_to_float(x[i]);
+        if (!isfinite(v)) return ORC_ERR_NONFINITE;
+        qx[i] = quantize_one(v, s);
+    }
+    return ORC_OK;
+}
+
 int oracle_act_quant(const uint16_t *x, int64_t numel, int8_t *qx, float *s_a)
 {
     float amax;
     int rc = oracle_act_absmax(x, numel, &amax);
     if (rc != ORC_OK) return rc;
-    amax = amax * 1.0f;              /* activation clip ratio 1.0 */
-    float s = amax / 127.0f;
-    *s_a = s;
-    for (int64_t i = 0; i < numel; ++i)
-        qx[i] = quantize_one(bf16_bits_to_float(x[i]), s);
-    return ORC_OK;
+    return oracle_act_quant_amax(x, numel, amax, qx, s_a);
 }
 
 /*

@@ -70,6 +70,7 @@ struct ConvArgs {
   int split;                  // per-sub-tile accumulator hand-off (one accumulator buffer, MS >= 2, SB >= 9 / G)
   int epi_bufs;               // staging buffers per epilogue warp (1 or 2)
   int carry;                  // 1: the input holds two carried frames before frame 0 (streamed chunk)
+  int halo_top;               // input rows above output row 0 (a row band's halo: 0 or 1)
   uint32_t a_stage_bytes;     // activation stage stride (1024-aligned)
   uint32_t a_box_bytes;       // bytes one activation box delivers
   uint32_t b_tap_bytes;       // weight rows this CTA loads per tap x 128 B
@@ -400,9 +401,9 @@ __global__ void __launch_bounds__(kConvThreads, 1)
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
           if (kPair) {
             tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * 128, c.w0 - 1,
-                             c.h0 - 1, frame, c.n);
+                             c.h0 - 1 + a.halo_top, frame, c.n);
           } else {
-            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1, frame,
+            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1 + a.halo_top, frame,
                         c.n);
           }
         }

@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __
                                                                   int64_t nvec,
                                                                   const uint16_t* __restrict__ xs,
                                                                   int64_t numel,
-                                                                  uint32_t* __restrict__ partial) {
+                                                                  uint32_t* __restrict__ partial,
+                                                                  uint32_t* amax_word) {
   __shared__ uint32_t red[kActThreads / 32];
   grid_dependents_launch();  // the quantiser may start its prologue
   uint32_t m[4] = {0u, 0u, 0u, 0u};
@@ -127,7 +128,13 @@ __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __
       m[0] = max(m[0], static_cast<uint32_t>(xs[k]) & 0x7FFFu);
   }
   const uint32_t mm = block_max_u32<kActThreads>(max(max(m[0], m[1]), max(m[2], m[3])), red);
-  if (threadIdx.x == 0) partial[blockIdx.x] = mm;
+  if (threadIdx.x == 0) {
+    if (amax_word) {
+      atomicMax(amax_word, mm);  // one maximum for the whole tensor (zeroed beforehand)
+    } else {
+      partial[blockIdx.x] = mm;
+    }
+  }
 }
 
 // 16 bf16 values (two 16-byte vectors) -> 16 codes (one 16-byte vector).

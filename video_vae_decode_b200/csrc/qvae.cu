@@ -279,12 +279,18 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
 
 // carry: xq holds T + 2 frames per batch item, the first two carried from
 // the previous chunk of a streamed video (output frames are the last T).
+// halo_top / halo_bot: xq holds H + halo_top + halo_bot rows, output row h
+// reading input rows h + halo_top - 1 .. h + halo_top + 1 (a row band).
 int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                 const int8_t* wq, const float* w_scale, const void* bias, void* out, int32_t* acc,
-                cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr) {
+                cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr, int halo_top = 0,
+                int halo_bot = 0) {
   int rc = check_shape(shape);
   if (rc) return rc;
-  if (carry && (static_cast<double>(shape->T + 2) * shape->H * shape->W * shape->Cin >= 1099511627776.0))
+  if (halo_top < 0 || halo_top > 1 || halo_bot < 0 || halo_bot > 1) return QVAE_ERR_ARG;
+  // the input tensor map's largest stride (one batch item) must fit 40 bits
+  if (static_cast<double>(shape->T + (carry ? 2 : 0)) * (shape->H + halo_top + halo_bot) * shape->W *
+          shape->Cin >= 1099511627776.0)
     return QVAE_ERR_SHAPE;
   const bool acc_mode = acc != nullptr;
   const qvae_shape& s = *shape;
@@ -305,12 +311,13 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   CUtensorMap tmap_x, tmap_w, tmap_out;
   {
     const cuuint64_t t_in = static_cast<cuuint64_t>(s.T) + (carry ? 2 : 0);
-    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W),
-                                static_cast<cuuint64_t>(s.H), t_in, static_cast<cuuint64_t>(s.N)};
+    const cuuint64_t h_in = static_cast<cuuint64_t>(s.H) + halo_top + halo_bot;
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W), h_in, t_in,
+                                static_cast<cuuint64_t>(s.N)};
     const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin),
                                    static_cast<cuuint64_t>(s.W) * s.Cin,
-                                   static_cast<cuuint64_t>(s.H) * s.W * s.Cin,
-                                   t_in * s.H * s.W * s.Cin};
+                                   h_in * s.W * s.Cin,
+                                   t_in * h_in * s.W * s.Cin};
     const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(qvae::kBoxW),
                                static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
     rc = encode_map(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims, strides, box, 5,
@@ -368,6 +375,7 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.split = t.split ? 1 : 0;
   a.epi_bufs = t.epi_bufs;
   a.carry = carry ? 1 : 0;
+  a.halo_top = halo_top;
   a.out_amax = acc_mode ? nullptr : out_amax;
   a.b_tap_bytes = t.b_tap_bytes;
   a.b_stage_bytes = t.b_stage_bytes;
@@ -527,7 +535,7 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   const int g1 = act_grid(numel, sms);
   uint32_t* partial = static_cast<uint32_t*>(ws);
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial);
+      static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial, nullptr);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
   const int g2 = quant_grid(numel, sms);
@@ -661,6 +669,46 @@ int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
                      static_cast<cudaStream_t>(stream));
 }
 
+int qvae_act_absmax(const void* x_bf16, int64_t numel, uint32_t* amax, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (numel < 0 || !amax) return QVAE_ERR_ARG;
+  if (numel > 0 && !x_bf16) return QVAE_ERR_ARG;
+  if (numel > 0 && !aligned16(x_bf16)) return QVAE_ERR_ALIGN;
+  QVAE_CUDA(cudaMemsetAsync(amax, 0, sizeof(uint32_t), st));
+  if (numel == 0) return QVAE_OK;
+  int dev, sms, rc;
+  if ((rc = current_device(&dev))) return rc;
+  if ((rc = sm_count(dev, &sms))) return rc;
+  qvae::act_absmax_kernel<<<act_grid(numel, sms), qvae::kActThreads, 0, st>>>(
+      static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, nullptr,
+      amax);
+  QVAE_CUDA(cudaGetLastError());
+  return QVAE_OK;
+}
+
+int qvae_act_quant_from_absmax(const void* x_bf16, int64_t numel, const uint32_t* amax, int8_t* xq,
+                               float* x_scale, void* stream) {
+  if (numel < 0 || !amax || !x_scale) return QVAE_ERR_ARG;
+  if (numel > 0 && (!x_bf16 || !xq)) return QVAE_ERR_ARG;
+  if (numel > 0 && (!aligned16(x_bf16) || !aligned16(xq))) return QVAE_ERR_ALIGN;
+  return launch_quant_from_amax(x_bf16, numel, amax, xq, x_scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int qvae_causal_conv3d_w8a8_band(const qvae_shape* shape, int32_t halo_top, int32_t halo_bot,
+                                 const int8_t* xq_band, const float* x_scale, const int8_t* wq_packed,
+                                 const float* w_scale, const void* bias_bf16, void* out_bf16, void* stream) {
+  return launch_conv(shape, xq_band, x_scale, wq_packed, w_scale, bias_bf16, out_bf16, nullptr,
+                     static_cast<cudaStream_t>(stream), false, nullptr, halo_top, halo_bot);
+}
+
+int qvae_causal_conv3d_w8a8_band_acc32(const qvae_shape* shape, int32_t halo_top, int32_t halo_bot,
+                                       const int8_t* xq_band, const int8_t* wq_packed, int32_t* acc,
+                                       void* stream) {
+  if (!acc) return QVAE_ERR_ARG;
+  return launch_conv(shape, xq_band, nullptr, wq_packed, nullptr, nullptr, nullptr, acc,
+                     static_cast<cudaStream_t>(stream), false, nullptr, halo_top, halo_bot);
+}
+
 int qvae_causal_conv3d_w8a8_carry(const qvae_shape* shape, const int8_t* xq_ext, const float* x_scale,
                                   const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
                                   void* out_bf16, void* stream) {
@@ -702,7 +750,8 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
   // Same two kernels as qvae_act_absmax_quant; every slot the second reads is
   // written by the first in this call, so nothing needs clearing.
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, st>>>(
-      static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, partial);
+      static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, partial,
+      nullptr);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
   const int g2 = quant_grid(numel, sms);

@@ -29,6 +29,8 @@ EXPORTS = (
     "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
     "qvae_act_absmax_quant_noalloc", "qvae_set_act_passes",
     "qvae_causal_conv3d_w8a8_carry", "qvae_causal_conv3d_w8a8_carry_acc32",
+    "qvae_act_absmax", "qvae_act_quant_from_absmax",
+    "qvae_causal_conv3d_w8a8_band", "qvae_causal_conv3d_w8a8_band_acc32",
 )
 
 
@@ -73,6 +75,12 @@ def lib():
             "qvae_causal_conv3d_w8a8_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_carry": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_carry_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
+            "qvae_act_absmax": ([p, i64, p, p], ctypes.c_int),
+            "qvae_act_quant_from_absmax": ([p, i64, p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_band": ([ctypes.POINTER(qvae_shape), i32, i32, p, p, p, p, p, p, p],
+                                             ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_band_acc32": ([ctypes.POINTER(qvae_shape), i32, i32, p, p, p, p],
+                                                   ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
             "qvae_decode_layers": ([ctypes.POINTER(qvae_layer), i32, p, sz, p], ctypes.c_int),
             "qvae_get_error": ([p], ctypes.c_int),
@@ -238,6 +246,44 @@ def conv_carry_acc32(xq_ext, wq_packed, Cout: int, stream=None):
     acc = torch.empty((N, T2 - 2, H, W, Cout), dtype=torch.int32, device=xq_ext.device)
     qvae_causal_conv3d_w8a8_carry_acc32(xq_ext, wq_packed, acc, stream)
     return acc
+
+
+def qvae_act_absmax(x: torch.Tensor, amax: torch.Tensor, stream=None) -> None:
+    """amax: a 4-byte device tensor (int32 or uint32) that receives max |x| as bf16 magnitude bits."""
+    _check("qvae_act_absmax", lib().qvae_act_absmax(_ptr(x), x.numel(), _ptr(amax), _stream(stream)))
+
+
+def qvae_act_quant_from_absmax(x: torch.Tensor, amax: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor,
+                               stream=None) -> None:
+    _check("qvae_act_quant_from_absmax",
+           lib().qvae_act_quant_from_absmax(_ptr(x), x.numel(), _ptr(amax), _ptr(xq), _ptr(x_scale),
+                                            _stream(stream)))
+
+
+def _band_shape(xq_band: torch.Tensor, halo_top: int, halo_bot: int, Cout: int) -> qvae_shape:
+    N, T, Hin, W, Cin = xq_band.shape
+    H = Hin - halo_top - halo_bot
+    if H < 0:
+        raise ValueError("a band holds its halo rows and its own")
+    return make_shape(N, T, H, W, Cin, Cout)
+
+
+def qvae_causal_conv3d_w8a8_band(xq_band: torch.Tensor, halo_top: int, halo_bot: int, x_scale: torch.Tensor,
+                                 wq_packed: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor],
+                                 out: torch.Tensor, stream=None) -> None:
+    shp = _band_shape(xq_band, halo_top, halo_bot, int(out.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_band",
+           lib().qvae_causal_conv3d_w8a8_band(ctypes.byref(shp), int(halo_top), int(halo_bot), _ptr(xq_band),
+                                              _ptr(x_scale), _ptr(wq_packed), _ptr(w_scale), _ptr(bias),
+                                              _ptr(out), _stream(stream)))
+
+
+def qvae_causal_conv3d_w8a8_band_acc32(xq_band: torch.Tensor, halo_top: int, halo_bot: int,
+                                       wq_packed: torch.Tensor, acc: torch.Tensor, stream=None) -> None:
+    shp = _band_shape(xq_band, halo_top, halo_bot, int(acc.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_band_acc32",
+           lib().qvae_causal_conv3d_w8a8_band_acc32(ctypes.byref(shp), int(halo_top), int(halo_bot),
+                                                    _ptr(xq_band), _ptr(wq_packed), _ptr(acc), _stream(stream)))
 
 
 def conv_acc32(xq, wq_packed, Cout: int, stream=None):
