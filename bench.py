@@ -83,11 +83,20 @@ def measured_peaks():
         return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def code_only(src: str) -> str:
+    """C/C++ source without comments and blank lines (comment edits keep the hash)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in src.splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def conv_source_hash():
+    """Hash of the convolution kernel's code (conv.cuh + ptx.cuh, comments stripped)."""
     h = hashlib.sha256()
     for f in ("conv.cuh", "ptx.cuh"):
-        with open(os.path.join(ROOT, "video_vae_decode_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "video_vae_decode_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

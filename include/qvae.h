@@ -25,6 +25,9 @@
  *     of time is reported later by qvae_get_error().
  *   - Layer geometry is fixed: 3x3x3 kernel, stride 1, causal temporal
  *     padding of 2 leading zero frames, spatial padding 1 ("same" size).
+ *     The streamed-chunk variant takes two carried frames in place of the
+ *     zero frames, the row-band variant halo rows in place of the top and
+ *     bottom padding.
  */
 #ifndef QVAE_H
 #define QVAE_H

@@ -24,7 +24,9 @@
 // absolute shared-memory address, so any line offset is a valid operand start:
 // the halo is loaded once and reused nine times.  Temporal taps that meet a
 // causal zero frame are skipped, not computed.  Weights come pre-packed in the
-// MMA's swizzled K-major layout and stream one tap at a time by 2-D TMA.
+// MMA's swizzled K-major layout and stream by 2-D TMA, G taps (1, or 3 = one
+// kernel row) per pipeline stage, so the MMA thread waits and commits once per
+// G taps.
 //
 // CTA pairs.  With kPair the kernel runs as 2-CTA clusters on the tensor
 // cores' cta_group::2 path: one MMA covers M = 256 (128 pixels in each CTA)
@@ -32,17 +34,26 @@
 // weight tile (NT/2 rows), so weight traffic and shared-memory reads per
 // multiply-add halve.  Every load of both CTAs is counted on the leader CTA's
 // barriers; the leader issues the MMAs and its commits arrive on the barriers
-// of both CTAs; each CTA's epilogue drains its own TMEM rows.
+// of both CTAs; each CTA's epilogue drains its own TMEM rows.  No TMA load
+// uses cluster multicast.
 //
-// Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 issues tcgen05.mma
-// (one thread) and owns the TMEM allocation, warps 2-5 run the epilogue:
-// tcgen05.ld of their 32 TMEM lanes, rescale + bias + bf16, staged through
-// shared memory and written with TMA stores.  Tiles are scheduled
-// persistently (static stride); with MS*NT <= 256 TMEM columns the
-// accumulator is double-buffered so the epilogue of one tile overlaps the
-// main loop of the next.
+// Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 issues
+// tcgen05.mma (one thread) and owns the TMEM allocation, warps 2-9 run the
+// epilogue (two per TMEM lane quarter): tcgen05.ld of their 32 TMEM lanes,
+// rescale + bias + bf16, staged through shared memory and written with TMA
+// stores.  Tiles are scheduled persistently (static stride).  With MS*NT <=
+// 256 TMEM columns the accumulator is double-buffered so the epilogue of one
+// tile overlaps the main loop of the next; with one buffer of several
+// sub-tiles, the sub-tiles are handed to the epilogue one by one (see
+// mma_issue_loop).
 // Launched as a programmatic dependent of the activation quantiser: the
 // prologue and the first weight loads overlap its tail.
+//
+// Variants of the same kernel (ConvArgs): a streamed chunk whose input holds
+// two carried frames in place of the causal zero frames (carry), a row band
+// whose input holds halo rows in place of the top / bottom padding
+// (halo_top), raw INT32 accumulators instead of the bf16 output (kAcc32), and
+// the maximum |output| accumulated for the next layer's quantiser (out_amax).
 #pragma once
 
 #include <cuda.h>
