@@ -410,3 +410,21 @@ def test_layer_carry_zero_history_equals_layer():
     ext = np.concatenate([np.zeros_like(xb[:, :2]), xb], axis=1)
     a, b = oracle.layer_carry(ext, wb, bb), oracle.layer(xb, wb, bb)
     assert a["s_a"] == b["s_a"] and np.array_equal(a["out"], b["out"])
+
+
+def test_epilogue_rounds_the_product_before_adding_the_bias():
+    # A bf16 tie met on B200: acc = 135 with this scale and bias gives
+    # y + b = -2.8405339e-07 exactly (0xb4988000), which rounds to even
+    # (0xb498).  A fused multiply-add (one rounding) lands at 0xb4988c80 and
+    # rounds to 0xb499: the oracle must keep the two roundings.
+    s_a = np.float32(1.0)
+    s_w = np.array([np.float32(3.3906315e-05)], dtype=np.float32)
+    bias = np.array([np.uint32(np.float32(-0.0045776367).view(np.uint32) >> 16)], dtype=np.uint16)
+    out = oracle.epilogue(np.array([[135]], dtype=np.int32), s_a, s_w, bias)
+    y = np.float32(np.float32(135.0) * np.float32(s_w[0] * s_a))
+    b = np.uint32(int(bias[0]) << 16).view(np.float32)
+    sep = np.float32(y + b)
+    assert sep.view(np.uint32) == 0xB4988000
+    fused = np.float32(135.0 * np.float64(s_w[0]) + np.float64(b))
+    assert fused.view(np.uint32) != sep.view(np.uint32)
+    assert int(out[0, 0]) == 0xB498
