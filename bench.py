@@ -31,6 +31,7 @@ DATASHEET_INT8_TOPS = 4500.0          # B200 dense INT8, NVIDIA datasheet
 INT8_PER_BF16 = 2.0                    # nominal dense INT8 : BF16 ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 10**6
+ARITHMETIC = "int8 x int8 products, int32 accumulation, fp32 rescale + bias, bf16 in and out"
 SPIN_CYCLES = 200_000                  # ~100 us of GPU spin ahead of each event-timed group
 
 
@@ -236,9 +237,10 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ops / (v * 1e12) * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/int32/f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
-        "config": {"workload": args.workload, "layer": layer_name(layer), "l2": "n/a (CPU)"},
+        "config": {"workload": args.workload, "layer": layer_name(layer), "l2": "n/a (CPU)",
+                   "arithmetic": ARITHMETIC},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -498,9 +500,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, f32 epilogue, bf16 io",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
-        "config": {"workload": args.workload, "layer": layer_name(layer),
+        "config": {"workload": args.workload, "layer": layer_name(layer), "arithmetic": ARITHMETIC,
                    "tiling": qvae.qvae_get_conv_tiling(s.N, s.T, s.H, s.W, s.Cin, s.Cout),
                    "l2": (f"inputs, codes, outputs and packed weights rotate over {n_sets} buffer sets "
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
@@ -608,9 +610,9 @@ def run_chain(args):
     line = {
         "metric": METRIC + ", layer chain", "value": ops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, f32 epilogue, bf16 io",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
-        "config": {"workload": args.workload, "chain": [layer_name(t) for t in tens],
+        "config": {"workload": args.workload, "chain": [layer_name(t) for t in tens], "arithmetic": ARITHMETIC,
                    "l2": f"{n_sets} buffer sets rotate ({n_sets * per_set / 2**20:.0f} MiB)",
                    "launch": "one CUDA graph replay per chain (qvae_decode_layers)", "ops": ops},
         "unchained_ms_per_step": ms_unchained,
