@@ -128,3 +128,20 @@ def test_tiling_choice_is_valid():
         qvae.qvae_set_conv_tiling(G=2)
     with pytest.raises(qvae.QvaeError):
         qvae.qvae_set_conv_tiling(MS=3, G=3)
+
+
+def test_tiling_choice_is_valid_over_the_supported_shapes():
+    """The cost model picks a launchable tiling for every shape the kernel accepts."""
+    chans = (32, 64, 96, 128, 160, 192, 256, 384, 512)
+    for Cin in chans:
+        for Cout in chans:
+            for H, W in ((1, 1), (7, 33), (16, 8), (33, 7), (128, 128), (517, 300)):
+                for T in (1, 3):
+                    t = qvae.qvae_get_conv_tiling(1, T, H, W, Cin, Cout)
+                    assert 1 <= t["MS"] <= 4 and t["MS"] * t["NT"] <= 512 and t["mode"] in (1, 2)
+                    assert Cout % t["NT"] == 0 and t["NT"] % 32 == 0 and t["NT"] <= 256
+                    assert 1 <= t["SA"] <= 12 and 1 <= t["SB"] <= 12
+                    assert t["G"] == 1 or (t["G"] == 3 and t["MS"] <= 2)
+                    assert t["acc_buffers"] == (2 if 2 * t["MS"] * t["NT"] <= 512 else 1)
+                    rows = 16 * t["MS"] * t["mode"]
+                    assert t["ctas"] == T * -(-H // rows) * -(-W // 8) * (Cout // t["NT"]) * t["mode"]
