@@ -388,9 +388,14 @@ def run_ours(args):
     # One CUDA graph per buffer set holds that set's step (the three kernels,
     # with their programmatic launch dependencies): a replay costs the host one
     # call, so the timed loop measures the device, not the Python launch path.
+    # First call of the layer in this process (tiling choice, tensor-map
+    # encoding, kernel attributes and module load included), host wall clock.
+    torch.cuda.synchronize()
+    t_first = time.perf_counter()
+    step(sets[0])
+    torch.cuda.synchronize()
+    first_call_ms = (time.perf_counter() - t_first) * 1e3
     if args.launch == "graph":
-        step(sets[0])  # first call outside capture: one-time attribute setup
-        torch.cuda.synchronize()
         graphs = []
         for st in sets:
             g = torch.cuda.CUDAGraph()
@@ -445,6 +450,25 @@ def run_ours(args):
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     act_ms = [a.elapsed_time(m) for a, m, _ in ev]
+
+    # A resolution switch: the first call of the same layer at the spatial size
+    # scaled by 840/1024 (the pages' switch from 1024x1024 to 840x1256 output),
+    # in this warm process; nothing is compiled per shape.
+    Hs, Ws = max(1, (s.H * 840) // 1024), max(1, (s.W * 1256) // 1024)
+    xs = torch.randn((s.N, s.T, Hs, Ws, s.Cin), device=dev).to(torch.bfloat16)
+    xqs = torch.empty(xs.shape, dtype=torch.int8, device=dev)
+    scs = torch.empty(1, dtype=torch.float32, device=dev)
+    wss = torch.empty(qvae.qvae_act_workspace_bytes(xs.numel()), dtype=torch.uint8, device=dev)
+    outs = torch.empty((s.N, s.T, Hs, Ws, s.Cout), dtype=torch.bfloat16, device=dev)
+    switch_ms = []
+    for _ in range(2):                            # first call, then the same call warm
+        torch.cuda.synchronize()
+        t_sw = time.perf_counter()
+        qvae.qvae_act_absmax_quant(xs, xqs, scs, wss, stream)
+        qvae.qvae_causal_conv3d_w8a8(xqs, scs, packed0, s_w, b, outs, stream)
+        torch.cuda.synchronize()
+        switch_ms.append((time.perf_counter() - t_sw) * 1e3)
+    del xs, xqs, wss, outs
     conv_ms = [m.elapsed_time(z) for _, m, z in ev]
 
     # ---- end to end: pinned host input -> device -> layer -> pinned host output.
@@ -514,6 +538,15 @@ def run_ours(args):
         "ms_per_layer": {"step": ms_per_step, "act_absmax_quant": statistics.mean(act_ms),
                          "conv": conv_mean, "conv_median": statistics.median(conv_ms)},
         "conv_tops": conv_tops,
+        "act_gbs": {"moved_5B": 5 * layer.x.numel() / (statistics.mean(act_ms) * 1e-3) / 1e9,
+                    "algorithmic_3B": 3 * layer.x.numel() / (statistics.mean(act_ms) * 1e-3) / 1e9,
+                    "note": "activation passes: 5 B per element moved (bf16 read twice, int8 written; "
+                            "the second read hits L2 when x fits), 3 B algorithmic; measured copy "
+                            "bandwidth 6557 GB/s"},
+        "first_call_ms": {"process_first": first_call_ms,
+                          "resolution_switch": {"shape": f"{Hs}x{Ws}", "first": switch_ms[0],
+                                                "warm": switch_ms[1]},
+                          "note": "host wall clock, act + conv with a device synchronise"},
         "pct_datasheet_int8_peak": 100.0 * conv_tops / DATASHEET_INT8_TOPS,
         "roofline": {"bound": "tensor", "achieved": conv_tops, "peak": peak, "unit": "TOPS",
                      "frac": conv_tops / peak, "traffic": traffic,
