@@ -16,14 +16,19 @@
  *     ratios are 1.0, channels_last layout;
  *   - opening paragraph: the layer is a CausalConv3d (implicit-GEMM lowering
  *     is only how the kernel evaluates it; the result is the plain sum below).
- * Readings where the page is silent (each listed in the design doc):
+ * Readings where the page is silent:
  *   - activation scale is per tensor; scale = absmax / 127 (IEEE fp32 divide);
  *   - code = clamp(rint(v / scale), -127, 127), rint = round half to even,
  *     v / scale an IEEE fp32 divide; absmax == 0 gives scale 0 and all codes 0;
  *   - causal padding is two leading zero frames (kernel slice kt = 2 meets
  *     frame t, kt = 0 meets frame t - 2), spatial padding 1, stride 1, 3x3x3;
  *   - epilogue: y = float(acc) * (s_a * s_w[co]), then y + float(bias[co]) as
- *     a separate add (no fused multiply-add), then bf16 round-to-nearest-even.
+ *     a separate add (no fused multiply-add), then bf16 round-to-nearest-even;
+ *   - streamed temporal decode (the release note names the Wan VAE; chunking
+ *     is a reading): a chunk's input carries the previous chunk's last two
+ *     input frames in place of the zero frames, quantised with the chunk;
+ *   - row bands: codes of every band are taken with the whole image's
+ *     maximum (oracle_act_quant_amax), so bands reproduce the whole image.
  *
  * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -shared -fPIC (see build.py).
  */
