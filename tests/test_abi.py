@@ -145,3 +145,33 @@ def test_tiling_choice_is_valid_over_the_supported_shapes():
                     assert t["acc_buffers"] == (2 if 2 * t["MS"] * t["NT"] <= 512 else 1)
                     rows = 16 * t["MS"] * t["mode"]
                     assert t["ctas"] == T * -(-H // rows) * -(-W // 8) * (Cout // t["NT"]) * t["mode"]
+
+
+def test_stream_band_and_split_activation_argument_checks():
+    L = qvae.lib()
+    ok = qvae.make_shape(1, 2, 8, 8, 64, 64)
+    bad = qvae.make_shape(1, 2, 8, 8, 48, 64)
+    # streamed chunk (two carried frames)
+    assert L.qvae_causal_conv3d_w8a8_carry(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                           None) == qvae.QVAE_ERR_SHAPE
+    assert L.qvae_causal_conv3d_w8a8_carry(ctypes.byref(ok), FAKE, None, FAKE, FAKE, None, FAKE,
+                                           None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_causal_conv3d_w8a8_carry_acc32(ctypes.byref(ok), FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+    # row band: halos of 0 or 1 rows only
+    for ht, hb in ((2, 0), (0, 2), (-1, 0)):
+        assert L.qvae_causal_conv3d_w8a8_band(ctypes.byref(ok), ht, hb, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                              None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_causal_conv3d_w8a8_band(ctypes.byref(ok), 1, 1, None, FAKE, FAKE, FAKE, None, FAKE,
+                                          None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_causal_conv3d_w8a8_band(ctypes.byref(ok), 1, 1, FAKE_ODD, FAKE, FAKE, FAKE, None, FAKE,
+                                          None) == qvae.QVAE_ERR_ALIGN
+    assert L.qvae_causal_conv3d_w8a8_band_acc32(ctypes.byref(ok), 0, 0, FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+    # the two activation steps apart
+    assert L.qvae_act_absmax(FAKE, -1, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_absmax(FAKE, 100, None, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_absmax(None, 100, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_absmax(FAKE_ODD, 100, FAKE, None) == qvae.QVAE_ERR_ALIGN
+    assert L.qvae_act_quant_from_absmax(FAKE, 100, None, FAKE, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, None, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, FAKE_ODD, FAKE, None) == qvae.QVAE_ERR_ALIGN
