@@ -428,3 +428,37 @@ def test_epilogue_rounds_the_product_before_adding_the_bias():
     fused = np.float32(135.0 * np.float64(s_w[0]) + np.float64(b))
     assert fused.view(np.uint32) != sep.view(np.uint32)
     assert int(out[0, 0]) == 0xB498
+
+
+# ------------------------------------------- property tests against a library conv
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+def _torch_conv(qx_padded_t, qw, pad_hw=1):
+    """float64 conv3d of codes already padded in time; spatial zero padding 1."""
+    x = torch.from_numpy(qx_padded_t.astype(np.float64)).permute(0, 4, 1, 2, 3)   # N C T H W
+    w = torch.from_numpy(qw.astype(np.float64))                                     # Co Ci kt kh kw
+    y = torch.nn.functional.conv3d(x, w, padding=(0, pad_hw, pad_hw))
+    return y.permute(0, 2, 3, 4, 1).numpy()
+
+
+@settings(max_examples=25, deadline=None)
+@given(N=st.integers(1, 2), T=st.integers(1, 4), H=st.integers(1, 6), W=st.integers(1, 6),
+       Cin=st.integers(1, 6), Cout=st.integers(1, 4), seed=st.integers(0, 2**31 - 1))
+def test_conv_acc_matches_a_library_conv(N, T, H, W, Cin, Cout, seed):
+    rng = np.random.default_rng(seed)
+    qx = rng.integers(-127, 128, size=(N, T, H, W, Cin), dtype=np.int8)
+    qw = rng.integers(-127, 128, size=(Cout, Cin, 3, 3, 3), dtype=np.int8)
+    padded = np.concatenate([np.zeros((N, 2, H, W, Cin), np.int8), qx], axis=1)   # two causal zero frames
+    assert np.array_equal(oracle.conv_acc(qx, qw), _torch_conv(padded, qw).astype(np.int64))
+
+
+@settings(max_examples=25, deadline=None)
+@given(T=st.integers(1, 3), H=st.integers(1, 5), W=st.integers(1, 5), Cin=st.integers(1, 5),
+       Cout=st.integers(1, 3), seed=st.integers(0, 2**31 - 1))
+def test_conv_acc_carry_matches_a_library_conv(T, H, W, Cin, Cout, seed):
+    rng = np.random.default_rng(seed)
+    ext = rng.integers(-127, 128, size=(1, T + 2, H, W, Cin), dtype=np.int8)      # carried frames first
+    qw = rng.integers(-127, 128, size=(Cout, Cin, 3, 3, 3), dtype=np.int8)
+    assert np.array_equal(oracle.conv_acc_carry(ext, qw), _torch_conv(ext, qw).astype(np.int64))
