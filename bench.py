@@ -7,10 +7,17 @@ would).  Default workload: the decoder top-stage layer for a 1024x1024 image
 (Cin = Cout = 384, 128x128 latent, T = 1, 1% outliers at +-8).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+                    [--layer I] [--chunk C | --bands B] [--chain I,J] [--launch graph|stream]
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank decodes its
 own independently seeded layer (weak scaling, no collective on the data
 path); the value is the ops of all ranks over the slowest rank's time.
+
+Other modes of the same measurement (one GPU): --chunk C decodes a
+multi-frame layer as a stream of C-frame chunks carrying two frames each;
+--bands B decodes one image layer in B row bands (tiled decode); --chain I,J
+runs consecutive layers of a workload through qvae_decode_layers, each
+output feeding the next input.  --impl reference times the CPU oracle.
 """
 import argparse
 import hashlib
