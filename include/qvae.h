@@ -121,8 +121,9 @@ int qvae_act_absmax_quant(const void* x_bf16, int64_t numel, int8_t* xq, float* 
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.
- *   - The array holds 4096 partial maxima; a launch needing more (a GPU with
- *     more than 1024 SMs) returns QVAE_ERR_UNSUPPORTED with a message.
+ *   - The array holds 4096 partial maxima, one per block of the absmax pass,
+ *     which launches at most 8 blocks per SM: a GPU with more than 512 SMs
+ *     would need more and gets QVAE_ERR_UNSUPPORTED with a message.
  *   - Every call on a device shares the one array and leaves the last call's
  *     partial maxima in it; nothing needs clearing because every slot a call
  *     reads is written earlier in the same call.  Calls that overlap on the
@@ -165,6 +166,15 @@ int qvae_act_quant_from_absmax(const void* x_bf16, int64_t numel, const uint32_t
  *   bias_bf16  [Cout] bf16, or NULL for no bias.
  *   out_bf16   [N][T][H][W][Cout] bf16, written.
  * Needs Cin % 32 == 0, Cout % 32 == 0; sizes with N*T*H*W == 0 do nothing.
+ * Ordering: the convolution is launched as a programmatic dependent of the
+ * kernel before it on the stream (its set-up overlaps that kernel's tail) and
+ * starts loading wq_packed before it waits for that kernel; xq, x_scale,
+ * w_scale and bias are read only after the wait.  So wq_packed must not be
+ * written by the kernel launched immediately before this call on the same
+ * stream.  qvae_quantize_weights keeps this true for its own output (it ends
+ * with an empty kernel); copies (cudaMemcpyAsync) and anything with a kernel
+ * in between are safe.  The same holds for every convolution entry point
+ * below and for qvae_decode_layers.
  */
 int qvae_causal_conv3d_w8a8(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                             const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
@@ -299,17 +309,6 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
  * A small cap makes each CTA walk several tiles of a small problem.
  */
 int qvae_set_conv_cta_limit(int32_t max_ctas);
-
-/*
- * Activation-pass override for tuning and tests (process-wide): 0 automatic
- * (currently two passes, which measured faster), 1 single pass whenever the
- * tensor fits in one co-resident grid's registers
- * (about 9.7 M values on a 148-SM B200; each thread holds up to 64 values,
- * the CTAs exchange partial maxima through a bounded grid barrier in the
- * workspace, x is read once), 2 always two passes (absmax, then quantise).
- * Both give identical codes and scale.
- */
-int qvae_set_act_passes(int32_t mode);
 
 /* The tiling the next convolution of this shape would use: out[0..7] = MS,
  * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G. */

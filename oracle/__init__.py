@@ -48,6 +48,10 @@ def lib():
         L.oracle_epilogue.restype = None
         L.oracle_f32_to_bf16.argtypes = [f32]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.oracle_conv_bf16.argtypes = [p, p, p, i64, i64, i64, i64, i32, i32, p, p]
+        L.oracle_conv_bf16.restype = ctypes.c_int
+        L.oracle_f64_to_bf16.argtypes = [p, i64, p]
+        L.oracle_f64_to_bf16.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -192,3 +196,33 @@ def layer(x_bits, w_bits, bias_bits=None):
     acc = conv_acc(qx, qw)
     out = epilogue(acc, s_a, s_w, bias_bits)
     return {"qw": qw, "s_w": s_w, "qx": qx, "s_a": s_a, "acc": acc, "out": out}
+
+
+def conv_bf16(x_bits, w_bits, bias_bits=None):
+    """Native-precision causal conv, exact: returns (y float64, s_abs float64), both
+    [N,T,H,W,Cout]; y = bias + sum of x*w, s_abs = |bias| + sum of |x*w|."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    N, T, H, W, Cin = x.shape
+    Cout = w.shape[0]
+    assert w.shape == (Cout, Cin, 3, 3, 3)
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    y = np.empty((N, T, H, W, Cout), dtype=np.float64)
+    s_abs = np.empty_like(y)
+    _check(lib().oracle_conv_bf16(_ptr(x), _ptr(w), _ptr(b), N, T, H, W, Cin, Cout, _ptr(y), _ptr(s_abs)),
+           "conv_bf16")
+    return y, s_abs
+
+
+def f64_to_bf16(values):
+    """Round float64 values to bf16 bits once (nearest, ties to even)."""
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().oracle_f64_to_bf16(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def layer_bf16(x_bits, w_bits, bias_bits=None):
+    """A native-precision layer: exact sum, then one rounding to bf16."""
+    y, s_abs = conv_bf16(x_bits, w_bits, bias_bits)
+    return {"y": y, "s_abs": s_abs, "out": f64_to_bf16(y)}

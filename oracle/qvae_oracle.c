@@ -28,7 +28,10 @@
  *     is a reading): a chunk's input carries the previous chunk's last two
  *     input frames in place of the zero frames, quantised with the chunk;
  *   - row bands: codes of every band are taken with the whole image's
- *     maximum (oracle_act_quant_amax), so bands reproduce the whole image.
+ *     maximum (oracle_act_quant_amax), so bands reproduce the whole image;
+ *   - native-precision layers (the two the Aggressive preset keeps): the
+ *     exact convolution of the bf16 values plus bias, rounded once to bf16
+ *     (oracle_conv_bf16, oracle_f64_to_bf16).
  *
  * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -shared -fPIC (see build.py).
  */
@@ -271,6 +274,102 @@ void oracle_epilogue(const int32_t *acc, int64_t M, int32_t Cout, float s_a,
             y = y + b;
             out[m * Cout + co] = float_to_bf16_bits(y);
         }
+}
+
+/*
+ * Native-precision layer.  The release note's Aggressive preset quantises 26
+ * of the 28 decoder convolutions and keeps two (decoder.upsamples.14.residual.2
+ * and .residual.6, the full-resolution 96-channel stage) in their original
+ * precision: the same causal 3x3x3 convolution evaluated on the bf16 values
+ * themselves.  Written out exactly:
+ *   y[n,t,h,w,co] = bias[co] + sum over kt,kh,kw,ci of
+ *                   x[n, t+kt-2, h+kh-1, w+kw-1, ci] * w[co, ci, kt, kh, kw]
+ * with zero outside the tensor, as for the quantised layer.  Each bf16 x bf16
+ * product has at most 16 significant bits, so it is exact in binary64, and
+ * the sum of at most 27*Cin + 1 such terms is kept in binary64 (its own
+ * rounding is below 2^-40 of the magnitudes involved).  s_abs receives the
+ * sum of the magnitudes of the same terms, bias included: the scale of the
+ * error that any binary32 evaluation of the sum can make.
+ * x: bf16 bits [N][T][H][W][Cin]; w: bf16 bits [Cout][Cin][3][3][3];
+ * bias: bf16 bits [Cout] or NULL; y, s_abs: [N][T][H][W][Cout].
+ */
+int oracle_conv_bf16(const uint16_t *x, const uint16_t *w, const uint16_t *bias, int64_t N,
+                     int64_t T, int64_t H, int64_t W, int32_t Cin, int32_t Cout, double *y,
+                     double *s_abs)
+{
+    if (N <= 0 || T <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0) return ORC_ERR_ARG;
+    const int64_t rows = N * T * H;
+    int rc_all = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t n = r / (T * H), t = (r / H) % T, h = r % H;
+        for (int64_t wo = 0; wo < W; ++wo)
+            for (int32_t co = 0; co < Cout; ++co) {
+                double b = bias ? (double)bf16_bits_to_float(bias[co]) : 0.0;
+                double sum = b, mag = fabs(b);
+                for (int kt = 0; kt < 3; ++kt) {
+                    int64_t ti = t + kt - 2;
+                    if (ti < 0) continue;
+                    for (int kh = 0; kh < 3; ++kh) {
+                        int64_t hi = h + kh - 1;
+                        if (hi < 0 || hi >= H) continue;
+                        for (int kw = 0; kw < 3; ++kw) {
+                            int64_t wi = wo + kw - 1;
+                            if (wi < 0 || wi >= W) continue;
+                            const uint16_t *xp = x + (((n * T + ti) * H + hi) * W + wi) * Cin;
+                            for (int32_t ci = 0; ci < Cin; ++ci) {
+                                int64_t widx = ((((int64_t)co * Cin + ci) * 3 + kt) * 3 + kh) * 3 + kw;
+                                double xv = (double)bf16_bits_to_float(xp[ci]);
+                                double wv = (double)bf16_bits_to_float(w[widx]);
+                                if (!isfinite(xv) || !isfinite(wv)) {
+#pragma omp atomic write
+                                    rc_all = ORC_ERR_NONFINITE;
+                                }
+                                sum += xv * wv;
+                                mag += fabs(xv * wv);
+                            }
+                        }
+                    }
+                }
+                int64_t o = (((n * T + t) * H + h) * W + wo) * Cout + co;
+                y[o] = sum;
+                s_abs[o] = mag;
+            }
+    }
+    return rc_all;
+}
+
+/*
+ * binary64 -> bf16, round to nearest, ties to even, in one rounding (going
+ * through binary32 first could round twice).  v finite and below the bf16
+ * overflow threshold.  The two bf16 neighbours of |v| are found by scaling
+ * with the spacing of bf16 values at that magnitude (8 significant bits, or
+ * the subnormal spacing 2^-133), both exact operations in binary64.
+ */
+static uint16_t double_to_bf16_bits(double v)
+{
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    int e;
+    frexp(a, &e);                       /* a in [2^(e-1), 2^e) */
+    int q = e - 8;
+    if (q < -133) q = -133;
+    double ulp = ldexp(1.0, q);
+    double k = floor(a / ulp);          /* a / ulp is exact (a power-of-two scaling) */
+    double lo = k * ulp, rem = a - lo;  /* both exact */
+    double pick;
+    if (rem < ulp / 2) pick = lo;
+    else if (rem > ulp / 2) pick = lo + ulp;
+    else pick = (fmod(k, 2.0) == 0.0) ? lo : lo + ulp;
+    float f = (float)pick;              /* exact: pick has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)((u >> 16) | (signbit(v) ? 0x8000u : 0u));
+}
+
+void oracle_f64_to_bf16(const double *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16_bits(v[i]);
 }
 
 int oracle_num_threads(void)

@@ -110,7 +110,8 @@ def _chain(q, shapes, passthrough=(), seed=31):
         w, b = t.w.cuda(), t.bias.cuda()
         packed, s_w = q.quantize_weights(w)
         out = torch.zeros((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
-        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=i not in passthrough))
+        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=i not in passthrough,
+                          w=w))
         weights.append((packed, s_w, b, s.Cout))
         x = out
     return specs, weights
@@ -126,6 +127,75 @@ def _layer_by_layer(q, specs, weights):
         xq, s_a = q.act_absmax_quant(sp["x"])
         outs.append(q.causal_conv3d_w8a8(xq, s_a, packed, s_w, b, Cout))
     return outs
+
+
+def _np_bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _check_chain_against_oracle(q, specs, weights):
+    """Every quantised layer of a qvae_decode_layers chain against the oracle.
+
+    The oracle chain starts from the first input alone: layer k's reference
+    input is the oracle's own output of layer k - 1 (the chain is bit-exact,
+    so the GPU's input bits must equal it).  For each k the chain is run
+    again on its first k + 1 layers, which leaves layer k's codes and scale
+    in the workspace (codes at offset 0, the scale after the largest input's
+    codes rounded up to 256 bytes); codes, scale, the INT32 accumulators of
+    those codes and the bf16 output are compared element by element.  Layer
+    k's output as the chain writes it when it also feeds layer k + 1 (with
+    the epilogue maximum) is checked as layer k + 1's input."""
+    import oracle
+    ref_in = _np_bits(specs[0]["x"])
+    for k, (sp, (packed, s_w, b, Cout)) in enumerate(zip(specs, weights)):
+        assert sp["quantized"]
+        for j in range(k + 1):
+            specs[j]["out"].fill_(0)
+        layers = q.make_layers(specs[:k + 1])
+        need = q.qvae_decode_workspace_bytes(layers)          # the layout follows these layers
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        q.qvae_decode_layers(layers, ws)
+        torch.cuda.synchronize()
+        assert q.qvae_get_error() == 0
+        x_bits = _np_bits(sp["x"])
+        assert np.array_equal(x_bits, ref_in), f"layer {k}: input differs from the oracle chain"
+        ref = oracle.layer(ref_in, _np_bits(sp["w"]), _np_bits(b))
+        numel = sp["x"].numel()
+        codes = ws[:numel].view(torch.int8).view(sp["x"].shape)
+        xq_bytes = need - 256 - q.qvae_act_workspace_bytes(1)
+        scale = ws[xq_bytes:xq_bytes + 4].view(torch.float32)
+        assert np.array_equal(codes.cpu().numpy(), ref["qx"]), f"layer {k}: codes differ"
+        assert scale.cpu().numpy().view(np.uint32)[0] == np.array([ref["s_a"]], np.float32).view(np.uint32)[0]
+        acc = q.conv_acc32(codes.contiguous(), packed, Cout)
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"]), f"layer {k}: accumulators differ"
+        got = _np_bits(sp["out"])
+        assert np.array_equal(got, ref["out"]), f"layer {k}: {np.count_nonzero(got != ref['out'])} outputs differ"
+        ref_in = ref["out"]
+
+
+def test_decode_chain_matches_the_oracle_at_every_layer(q):
+    # ragged sizes: the epilogue's maximum must skip rows and columns beyond the image
+    shapes = [synth.LayerShape(96, 192, 37, 21, T=2), synth.LayerShape(192, 192, 37, 21, T=2),
+              synth.LayerShape(192, 96, 37, 21, T=2)]
+    specs, weights = _chain(q, shapes)
+    _check_chain_against_oracle(q, specs, weights)
+
+
+def test_decode_chain_full_size_sweep_layers(q):
+    """384->192 then 192->192 at 512x512 (two layers of the 1024x1024 decoder sweep),
+    chained, every element against the oracle."""
+    tens = synth.draw_workload("decoder_sweep_1024", only=[2, 3])
+    x = tens[0].x.cuda()
+    specs, weights = [], []
+    for t in tens:
+        s = t.shape
+        w, b = t.w.cuda(), t.bias.cuda()
+        packed, s_w = q.quantize_weights(w)
+        out = torch.zeros((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
+        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=True, w=w))
+        weights.append((packed, s_w, b, s.Cout))
+        x = out
+    _check_chain_against_oracle(q, specs, weights)
 
 
 @pytest.mark.parametrize("passthrough", [(), (1,)])

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -24,10 +25,12 @@ namespace {
 using qvae::ConvArgs;
 
 thread_local std::string t_last_error;
-uint64_t g_wait_limit_ns = 2000000000ull;
-int32_t g_force[6] = {0, 0, 0, 0, 0, 0};  // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair), G
-int32_t g_cta_limit = 0;                  // cap on the conv grid (0 = one CTA per SM); tests and tuning
-int g_act_mode = 0;                   // 0 automatic (two passes), 1 single pass when it fits, 2 two passes
+// Process-wide settings, written by the control entry points and read by every
+// launch; atomics so that a setting changed on one host thread while another
+// launches is read whole (each value is independent).
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int32_t> g_force[6] = {};   // MS, NT, SA, SB, mode (1 single CTA, 2 CTA pair), G
+std::atomic<int32_t> g_cta_limit{0};    // cap on the conv grid (0 = one CTA per SM); tests and tuning
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
@@ -106,8 +109,8 @@ uint32_t smem_needed(const Tiling& t) {
 // sub-tile hand-off needs a whole chunk's stages).
 bool fit_stages(Tiling* t, int want_sb = 0) {
   if (g_force[2] || g_force[3]) {
-    t->SA = g_force[2] ? g_force[2] : 2;
-    t->SB = g_force[3] ? g_force[3] : 4;
+    t->SA = g_force[2] ? g_force[2].load() : 2;
+    t->SB = g_force[3] ? g_force[3].load() : 4;
     for (t->epi_bufs = 2; t->epi_bufs >= 1; --t->epi_bufs)
       if (smem_needed(*t) <= static_cast<uint32_t>(kSmemLimit)) return true;
     return false;
@@ -413,12 +416,14 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
       QVAE_CUDA(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg));
       g_max_clusters[dev] = std::max(n, 1);
     }
+    const int cta_limit = g_cta_limit.load();
     int clusters = std::min(t.num_tiles, g_max_clusters[dev]);
-    if (g_cta_limit > 0) clusters = std::max(1, std::min(clusters, g_cta_limit / 2));
+    if (cta_limit > 0) clusters = std::max(1, std::min(clusters, cta_limit / 2));
     grid = 2 * clusters;
   } else {
+    const int cta_limit = g_cta_limit.load();
     grid = std::min(t.num_tiles, sms);
-    if (g_cta_limit > 0) grid = std::min(grid, g_cta_limit);
+    if (cta_limit > 0) grid = std::min(grid, cta_limit);
   }
   QVAE_CUDA(launch_dependent(kernel, grid, qvae::kConvThreads, t.smem_bytes, stream, t.pair ? 2 : 1, tmap_x,
                              tmap_w, tmap_out, a));
@@ -428,11 +433,12 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
 // ------------------------------------------------------------- activations
 
 // Blocks of the absmax pass: enough for kAbsUnroll vectors per thread, at
-// most eight 256-thread blocks per SM (full occupancy).
+// most kActBlocksPerSm 256-thread blocks per SM (full occupancy).
+constexpr int kActBlocksPerSm = 8;
 int act_grid(int64_t numel, int sms) {
   const int64_t vec = numel / 8;
   const int64_t want = ceil_div(std::max<int64_t>(vec, 1), qvae::kActThreads * qvae::kAbsUnroll);
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms)));
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(kActBlocksPerSm) * sms)));
 }
 
 // Blocks of the quantise pass: kQuantUnroll 16-value groups per thread, at
@@ -440,76 +446,10 @@ int act_grid(int64_t numel, int sms) {
 int quant_grid(int64_t numel, int sms) {
   const int64_t nvec2 = numel / 16;
   const int64_t want = ceil_div(std::max<int64_t>(nvec2, 1), qvae::kActThreads * qvae::kQuantUnroll);
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 8LL * sms)));
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(kActBlocksPerSm) * sms)));
 }
 
-constexpr size_t kActWorkspace = 16384;  // 4096 partial maxima
-
-// Co-resident CTAs of the single-pass quantiser for V vectors per thread (0 if
-// it cannot launch), cached per device.
-int g_fused_blocks[kMaxDevices][5] = {};
-
-template <int V>
-int fused_blocks_per_sm() {
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qvae::act_absmax_quant_fused_kernel<V>,
-                                                    qvae::kFusedThreads, 0) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return n;
-}
-
-template <int V>
-cudaError_t launch_fused(int grid, cudaStream_t stream, const void* x, int64_t numel, void* ws, int8_t* xq,
-                         float* x_scale) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(qvae::kFusedThreads);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the grid barrier cannot deadlock
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qvae::act_absmax_quant_fused_kernel<V>, static_cast<const uint4*>(x),
-                            numel / 8, static_cast<const uint16_t*>(x), numel, static_cast<uint32_t*>(ws),
-                            reinterpret_cast<uint2*>(xq), xq, x_scale, g_wait_limit_ns * 2);
-}
-
-// Single pass when the tensor fits in one co-resident grid's registers
-// (up to 8 vectors of 8 values per thread); returns false to use two passes.
-bool try_fused_act(int dev, int sms, const void* x, int64_t numel, int8_t* xq, float* x_scale, void* ws,
-                   size_t ws_bytes, cudaStream_t stream, int* rc) {
-  const int64_t nvec = numel / 8;
-  static const int kV[5] = {1, 2, 4, 6, 8};
-  for (int vi = 0; vi < 5; ++vi) {
-    if (g_fused_blocks[dev][vi] == 0) {
-      const int b = vi == 0 ? fused_blocks_per_sm<1>() : vi == 1 ? fused_blocks_per_sm<2>()
-                  : vi == 2 ? fused_blocks_per_sm<4>() : vi == 3 ? fused_blocks_per_sm<6>()
-                  : fused_blocks_per_sm<8>();
-      g_fused_blocks[dev][vi] = b > 0 ? b : -1;
-    }
-    if (g_fused_blocks[dev][vi] < 0) continue;
-    const int64_t max_grid = static_cast<int64_t>(g_fused_blocks[dev][vi]) * sms;
-    const int64_t per_cta = static_cast<int64_t>(qvae::kFusedThreads) * kV[vi];
-    const int64_t grid = std::max<int64_t>(1, ceil_div(nvec, per_cta));
-    if (grid > max_grid) continue;
-    if (16 + 4 * grid > static_cast<int64_t>(ws_bytes)) return false;
-    cudaError_t e = cudaMemsetAsync(ws, 0, 16, stream);  // arrival counter and generation
-    if (e == cudaSuccess) {
-      const int g = static_cast<int>(grid);
-      e = vi == 0 ? launch_fused<1>(g, stream, x, numel, ws, xq, x_scale)
-        : vi == 1 ? launch_fused<2>(g, stream, x, numel, ws, xq, x_scale)
-        : vi == 2 ? launch_fused<4>(g, stream, x, numel, ws, xq, x_scale)
-        : vi == 3 ? launch_fused<6>(g, stream, x, numel, ws, xq, x_scale)
-                  : launch_fused<8>(g, stream, x, numel, ws, xq, x_scale);
-    }
-    *rc = (e == cudaSuccess) ? QVAE_OK : cuda_fail(e, "single-pass activation quantiser launch");
-    return true;
-  }
-  return false;
-}
+constexpr size_t kActWorkspace = 16384;  // 4096 partial maxima: enough for 512 SMs
 
 // zero_word (nullable): a device word the quantise pass sets to zero, for a
 // following convolution to accumulate its output maximum into.
@@ -527,12 +467,11 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   int dev, sms, rc;
   if ((rc = current_device(&dev))) return rc;
   if ((rc = sm_count(dev, &sms))) return rc;
-  // The single pass reads x once but needs a counter reset and a cooperative
-  // launch; measured slower than two passes on the decoder top-stage layer
-  // (6.3 M values), so it runs only when asked for.
-  if (g_act_mode == 1 && !zero_word && try_fused_act(dev, sms, x, numel, xq, x_scale, ws, ws_bytes, stream, &rc))
-    return rc;
   const int g1 = act_grid(numel, sms);
+  if (static_cast<size_t>(g1) * sizeof(uint32_t) > ws_bytes) {
+    t_last_error = "the activation workspace holds fewer partial maxima than this GPU's absmax pass writes";
+    return QVAE_ERR_UNSUPPORTED;
+  }
   uint32_t* partial = static_cast<uint32_t*>(ws);
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, stream>>>(
       static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial, nullptr);
@@ -579,7 +518,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // until the process exits.
 namespace {
 
-constexpr int kStaticPartialSlots = 4096;  // one 32-bit partial maximum per absmax CTA
+constexpr int kStaticPartialSlots = 4096;  // one 32-bit partial maximum per absmax CTA (512 SMs x 8)
 static __device__ __align__(256) uint32_t g_static_partials[kStaticPartialSlots];
 
 void* g_static_partials_addr[kMaxDevices] = {};
@@ -640,6 +579,8 @@ int qvae_quantize_weights(int32_t Cin, int32_t Cout, const void* w_bf16, int8_t*
   const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 65535));
   qvae::weight_pack_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(w_bf16), Cin, Cout,
                                                    nchunks, w_scale, wq_packed, wq_plain);
+  QVAE_CUDA(cudaGetLastError());
+  qvae::stream_fence_kernel<<<1, 32, 0, st>>>();  // see the convolution's early weight loads
   QVAE_CUDA(cudaGetLastError());
   return QVAE_OK;
 }
@@ -788,14 +729,22 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
     if (!L.quantized) continue;
     int rc = check_shape(&L.shape);
     if (rc) return rc;
-    Tiling t;
-    if ((rc = make_tiling(L.shape, &t))) return rc;  // the shape has a valid tiling
     if (!L.x || !L.out || !L.wq_packed || !L.w_scale) return QVAE_ERR_ARG;
     if (!aligned16(L.x) || !aligned16(L.out) || !aligned16(L.wq_packed)) return QVAE_ERR_ALIGN;
   }
   const size_t need = qvae_decode_workspace_bytes(layers, n);
   if (!workspace || workspace_bytes < need) return QVAE_ERR_ARG;
   if (!aligned16(workspace)) return QVAE_ERR_ALIGN;
+  if (n > 0) {
+    // every shape has a valid tiling on this GPU before anything is launched
+    int dev = 0, sms = 0, rc = current_device(&dev);
+    if (rc) return rc;
+    if ((rc = sm_count(dev, &sms))) return rc;
+    for (int32_t i = 0; i < n; ++i) {
+      Tiling t;
+      if (layers[i].quantized && (rc = make_tiling(layers[i].shape, &t, sms))) return rc;
+    }
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t xq_bytes = need - 256 - kActWorkspace;
   int8_t* xq = reinterpret_cast<int8_t*>(ws);
@@ -871,12 +820,6 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
 int qvae_set_conv_cta_limit(int32_t max_ctas) {
   if (max_ctas < 0) return QVAE_ERR_ARG;
   g_cta_limit = max_ctas;
-  return QVAE_OK;
-}
-
-int qvae_set_act_passes(int32_t mode) {
-  if (mode < 0 || mode > 2) return QVAE_ERR_ARG;
-  g_act_mode = mode;
   return QVAE_OK;
 }
 

@@ -27,7 +27,7 @@ EXPORTS = (
     "qvae_causal_conv3d_w8a8", "qvae_causal_conv3d_w8a8_acc32", "qvae_decode_workspace_bytes",
     "qvae_decode_layers", "qvae_get_error", "qvae_set_wait_limit_ns",
     "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
-    "qvae_act_absmax_quant_noalloc", "qvae_set_act_passes",
+    "qvae_act_absmax_quant_noalloc",
     "qvae_causal_conv3d_w8a8_carry", "qvae_causal_conv3d_w8a8_carry_acc32",
     "qvae_act_absmax", "qvae_act_quant_from_absmax",
     "qvae_causal_conv3d_w8a8_band", "qvae_causal_conv3d_w8a8_band_acc32",
@@ -89,7 +89,6 @@ def lib():
             "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
             "qvae_set_conv_cta_limit": ([i32], ctypes.c_int),
             "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), ctypes.POINTER(i32)], ctypes.c_int),
-            "qvae_set_act_passes": ([i32], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -341,10 +340,6 @@ def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0, G=0) -> None:
 
 def qvae_set_conv_cta_limit(max_ctas: int = 0) -> None:
     _check("qvae_set_conv_cta_limit", lib().qvae_set_conv_cta_limit(int(max_ctas)))
-
-
-def qvae_set_act_passes(mode: int = 0) -> None:
-    _check("qvae_set_act_passes", lib().qvae_set_act_passes(int(mode)))
 
 
 def qvae_get_conv_tiling(N, T, H, W, Cin, Cout) -> dict:
