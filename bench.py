@@ -1,22 +1,28 @@
-"""Benchmark of the W8A8 CausalConv3d layer on B200.
+"""Benchmark of the W8A8 CausalConv3d layers of the VAE decoder on B200.
 
-One step = the whole per-call path of one layer: activation absmax + INT8
-quantisation, then the implicit-GEMM convolution with its fused epilogue
-(weights are quantised and packed once, before timing, as a model load
-would).  Default workload: the decoder top-stage layer for a 1024x1024 image
-(Cin = Cout = 384, 128x128 latent, T = 1, 1% outliers at +-8).
+One step = the whole per-call path of every layer of the workload: for each
+layer the activation absmax + INT8 quantisation, then the implicit-GEMM
+convolution with its fused epilogue (weights are quantised and packed once,
+before timing, as a model load would).  Default workload: the six decoder
+layer shapes of a 1024x1024 decode (384->384 @128x128 and @256x256, 384->192
+and 192->192 @512x512, 192->96 and 96->96 @1024x1024, 1% outliers at +-8);
+its first layer is the same tensors as the single decoder top-stage layer
+(384->384, 128x128).  The line reports the whole sweep's TOPS and, per layer,
+ms, conv TOPS and the fraction of the INT8 tensor peak.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
-                    [--layer I] [--chunk C | --bands B] [--chain I,J] [--launch graph|stream]
+                    [--layer I] [--chunk C | --bands B | --split] [--chain I,J] [--launch graph|stream]
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank decodes its
-own independently seeded layer (weak scaling, no collective on the data
+own independently seeded layers (weak scaling, no collective on the data
 path); the value is the ops of all ranks over the slowest rank's time.
 
-Other modes of the same measurement (one GPU): --chunk C decodes a
-multi-frame layer as a stream of C-frame chunks carrying two frames each;
---bands B decodes one image layer in B row bands (tiled decode); --chain I,J
-runs consecutive layers of a workload through qvae_decode_layers, each
+Other modes (one layer, --layer I): --chunk C decodes a multi-frame layer as
+a stream of C-frame chunks carrying two frames each; --bands B decodes one
+image layer in B row bands (tiled decode); --split splits one image layer
+across the ranks by row bands (an all-reduce MAX of the activation maximum and
+one halo row to and from each neighbour over NCCL; strong scaling); --chain
+I,J runs consecutive layers of a workload through qvae_decode_layers, each
 output feeding the next input.  --impl reference times the CPU oracle.
 """
 import argparse
@@ -38,26 +44,30 @@ DATASHEET_INT8_TOPS = 4500.0          # B200 dense INT8, NVIDIA datasheet
 INT8_PER_BF16 = 2.0                    # nominal dense INT8 : BF16 ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 10**6
+HBM_GBS_MEASURED = 6557.0
 ARITHMETIC = "int8 x int8 products, int32 accumulation, fp32 rescale + bias, bf16 in and out"
+DATA = "synthetic (seeded stand-in for the decoder's latents and random-init weights)"
 SPIN_CYCLES = 200_000                  # ~100 us of GPU spin ahead of each event-timed group
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decoder_top_384_128x128")
-    ap.add_argument("--layer", type=int, default=0, help="layer index inside the workload")
+    ap.add_argument("--workload", default="decoder_sweep_1024")
+    ap.add_argument("--layer", type=int, default=-1, help="one layer of the workload (-1: all of them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=18.0)
     ap.add_argument("--chunk", type=int, default=0,
                     help="decode a multi-frame layer as a stream of chunks of this many frames, each "
                          "carrying the previous chunk's last two input frames (0: whole layer at once)")
     ap.add_argument("--bands", type=int, default=0,
                     help="decode one image layer in this many row bands (tiled decode: whole-image "
                          "absmax, then per band quantise + band convolution)")
+    ap.add_argument("--split", action="store_true",
+                    help="split one image layer across the ranks by row bands (strong scaling)")
     ap.add_argument("--chain", default="",
                     help="comma-separated consecutive layers of the workload run as one qvae_decode_layers "
                          "chain, each output feeding the next input (one GPU)")
@@ -67,7 +77,7 @@ def parse():
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
-    """Each rank decodes its own independently seeded layer (weak scaling)."""
+    """Each rank decodes its own independently seeded layers (weak scaling)."""
     return base_seed + rank
 
 
@@ -108,19 +118,30 @@ def conv_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per conv launch from the committed ncu summary, if it still
-    describes the current kernel source (else None)."""
+def profiled_traffic(key):
+    """DRAM bytes per conv launch of one layer from the committed ncu summaries,
+    if they still describe the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "conv_traffic.json")
     try:
         with open(path) as fh:
             d = json.load(fh)
     except (OSError, ValueError):
         return None
-    e = d.get(workload)
+    e = d.get(key)
     if not e or e.get("kernel_sha") != conv_source_hash():
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 class ClockSampler:
@@ -175,55 +196,86 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def layer_name(layer):
+    s = layer.shape
+    return f"{s.Cin}->{s.Cout} @{s.H}x{s.W} T={s.T} N={s.N}"
+
+
+def pick_layers(args):
+    from video_vae_decode_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    idx = list(range(len(wl.layers))) if args.layer < 0 else [args.layer]
+    return wl, idx
+
+
 # ------------------------------------------------------------- CPU baseline
 
-def oracle_baseline(layer, seconds):
-    """Time the CPU oracle on a bounded sample of the layer: the activation
+def oracle_sample(layer, seconds, threads=None):
+    """Time the CPU oracle on a bounded sample of one layer: the activation
     quantisation over the whole tensor (its time scaled to the sampled share)
-    plus the convolution and epilogue of a seeded subset of output pixels."""
+    plus the convolution and epilogue of a seeded subset of output pixels.
+    Returns (ops, seconds, description)."""
     import numpy as np
     import oracle
     from video_vae_decode_b200 import synth
 
     s = layer.shape
-    xb, wb, bb = synth.bits(layer.x), synth.bits(layer.w), synth.bits(layer.bias)
-    qw, s_w = oracle.quantize_weights(wb)                  # one-time, not timed (as on the GPU)
-    t0 = time.perf_counter()
-    qx, s_a = oracle.act_quant(xb)
-    t_act = time.perf_counter() - t0
-    total_px = s.N * s.T * s.H * s.W
-    rng = np.random.default_rng(0)
+    if threads:
+        oracle.set_num_threads(threads)
+    try:
+        xb, wb, bb = synth.bits(layer.x), synth.bits(layer.w), synth.bits(layer.bias)
+        qw, s_w = oracle.quantize_weights(wb)              # one-time, not timed (as on the GPU)
+        t0 = time.perf_counter()
+        qx, s_a = oracle.act_quant(xb)
+        t_act = time.perf_counter() - t0
+        total_px = s.N * s.T * s.H * s.W
+        rng = np.random.default_rng(0)
 
-    def points(n):
-        return np.stack([rng.integers(0, s.N, n), rng.integers(0, s.T, n), rng.integers(0, s.H, n),
-                         rng.integers(0, s.W, n)], 1).astype(np.int64)
+        def run(n):
+            pts = np.stack([rng.integers(0, s.N, n), rng.integers(0, s.T, n), rng.integers(0, s.H, n),
+                            rng.integers(0, s.W, n)], 1).astype(np.int64)
+            t = time.perf_counter()
+            acc = oracle.conv_acc_points(qx, qw, pts)
+            oracle.epilogue(acc, s_a, s_w, bb)
+            return time.perf_counter() - t, pts
 
-    def run(n):
-        pts = points(n)
-        t = time.perf_counter()
-        acc = oracle.conv_acc_points(qx, qw, pts)
-        oracle.epilogue(acc, s_a, s_w, bb)
-        return time.perf_counter() - t, pts
-
-    probe = 32
-    dt, _ = run(probe)
-    n = int(min(total_px, max(probe, probe * seconds / max(dt, 1e-6))))
-    dt, pts = run(n)
-    taps = np.array([min(t + 1, 3) for t in range(s.T)])[pts[:, 1]]
-    ops = float(np.sum(2.0 * s.Cin * s.Cout * 9 * taps))
-    t_total = dt + t_act * n / total_px
-    return {
-        "value": ops / t_total / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-        "sample": (f"{n} of {total_px} output pixels (all {s.Cout} channels) of {layer_name(layer)}: "
-                   f"conv + epilogue {dt:.2f} s, plus the whole-tensor act quantisation "
-                   f"({t_act:.3f} s) scaled by {n}/{total_px}"),
-        "seconds": t_total,
-    }
+        probe = 16
+        dt, _ = run(probe)
+        n = int(min(total_px, max(probe, probe * seconds / max(dt, 1e-6))))
+        dt, pts = run(n)
+        taps = np.array([min(t + 1, 3) for t in range(s.T)])[pts[:, 1]]
+        ops = float(np.sum(2.0 * s.Cin * s.Cout * 9 * taps))
+        t_total = dt + t_act * n / total_px
+        desc = (f"{n} of {total_px} output pixels of {layer_name(layer)}: conv + epilogue {dt:.2f} s, "
+                f"plus the whole-tensor act quantisation ({t_act:.3f} s) scaled by {n}/{total_px}")
+        return ops, t_total, desc
+    finally:
+        if threads:
+            oracle.set_num_threads(os.cpu_count() or 1)
 
 
-def layer_name(layer):
-    s = layer.shape
-    return f"{s.Cin}->{s.Cout} @{s.H}x{s.W} T={s.T} N={s.N}"
+def oracle_baseline(layers, seconds, one_thread=True):
+    """The oracle over a bounded sample of every layer of the workload (about
+    `seconds` of CPU work in all), plus a 1-thread rate on the decoder
+    top-stage layer and the 96-channel 64x64 layer."""
+    import oracle
+    from video_vae_decode_b200 import synth
+    ops = tsec = 0.0
+    parts = []
+    for layer in layers:
+        o, t, d = oracle_sample(layer, seconds / len(layers))
+        ops += o
+        tsec += t
+        parts.append(d)
+    out = {"value": ops / tsec / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": "; ".join(parts), "cpu_model": cpu_model(), "seconds": tsec}
+    if one_thread:
+        single = {}
+        for name in ("decoder_top_384_128x128", "single_96_64x64"):
+            o, t, d = oracle_sample(synth.draw_workload(name)[0], 1.5, threads=1)
+            single[name] = {"value": o / t / 1e12, "unit": UNIT, "sample": d}
+        out["one_thread"] = single
+    return out
 
 
 def run_reference(args):
@@ -231,25 +283,25 @@ def run_reference(args):
     if rank != 0:
         return 0
     from video_vae_decode_b200 import synth
-    layer = synth.draw_workload(args.workload, only=[args.layer])[0]
+    wl, idx = pick_layers(args)
+    layers = synth.draw_workload(args.workload, only=idx)
     steps = []
-    budget = min(args.cpu_seconds, max(1.0, 150.0 / max(args.steps + min(args.warmup, 1), 1)))
+    budget = min(args.cpu_seconds, max(2.0, 150.0 / max(args.steps + min(args.warmup, 1), 1)))
     if args.warmup:
-        oracle_baseline(layer, min(budget, 1.0))          # untimed: page in the library and data
+        oracle_baseline(layers, min(budget, 2.0), one_thread=False)   # untimed: page in library and data
     for _ in range(args.steps):
-        steps.append(oracle_baseline(layer, budget))
+        steps.append(oracle_baseline(layers, budget, one_thread=False))
     v = statistics.median(r["value"] for r in steps)
     last = steps[-1]
-    ops = layer.shape.ops()
+    ops = sum(l.shape.ops() for l in layers)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ops / (v * 1e12) * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
-        "config": {"workload": args.workload, "layer": layer_name(layer), "l2": "n/a (CPU)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": DATA,
+        "config": {"workload": args.workload, "layers": [layer_name(l) for l in layers], "l2": "n/a (CPU)",
                    "arithmetic": ARITHMETIC},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
-                         "sample": last["sample"]},
+                         "sample": last["sample"], "cpu_model": last["cpu_model"]},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -257,6 +309,135 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- GPU arm
+
+def int8_cublas_tops(dev, n=8192, iters=20):
+    """Dense INT8 GEMM rate of the library GEMM (torch._int_mm, cuBLAS) at n^3: a
+    measured INT8 reference beside the bf16-derived peak.  None if unavailable."""
+    import torch
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        return 2.0 * n ** 3 * iters / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+class LayerJob:
+    """Buffers and launches of one layer (plain, streamed chunks or row bands)."""
+
+    def __init__(self, layer, dev, stream, qvae, args, single):
+        import torch
+        self.layer, self.s, self.stream, self.qvae = layer, layer.shape, stream, qvae
+        s = self.s
+        self.w, self.b = layer.w.to(dev), layer.bias.to(dev)
+        self.packed0, self.s_w = qvae.quantize_weights(self.w)   # once, as at model load
+        self.chunk = args.chunk if (single and args.chunk > 0 and s.T > args.chunk) else 0
+        if self.chunk and s.N != 1:
+            raise SystemExit("--chunk streams one video (N = 1)")
+        self.nb = args.bands if (single and args.bands > 1) else 0
+        if self.nb and s.N * s.T != 1:
+            raise SystemExit("--bands decodes one image (N = T = 1)")
+        if self.nb and self.chunk:
+            raise SystemExit("--bands and --chunk do not combine")
+        self.starts = list(range(0, s.T, self.chunk)) if self.chunk else [0]
+        self.dev = dev
+
+    def set_bytes(self):
+        s = self.s
+        return self.layer.x.numel() * 3 + s.pixels * s.Cout * 2 + self.packed0.numel()
+
+    def make_set(self):
+        import torch
+        qvae, s, dev = self.qvae, self.s, self.dev
+        st = dict(x=self.layer.x.to(dev), xq=torch.empty(self.layer.x.shape, dtype=torch.int8, device=dev),
+                  x_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                  ws=torch.empty(qvae.qvae_act_workspace_bytes(self.layer.x.numel()), dtype=torch.uint8,
+                                 device=dev),
+                  out=torch.empty((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device=dev),
+                  packed=self.packed0.clone())
+        if self.chunk:
+            # chunk k covers frames [kC, kC + C); its input is the view x[:, kC - 2 : kC + C]
+            # (the two frames before it carried), quantised as one tensor
+            st["chunks"] = []
+            for k, t0 in enumerate(self.starts):
+                t1 = min(t0 + self.chunk, s.T)
+                xv = st["x"][:, (t0 - 2 if k else 0):t1]
+                st["chunks"].append(dict(
+                    k=k, x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
+                    x_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                    ws=torch.empty(qvae.qvae_act_workspace_bytes(xv.numel()), dtype=torch.uint8, device=dev),
+                    out=st["out"][:, t0:t1]))
+            del st["xq"]
+        if self.nb:
+            from video_vae_decode_b200 import bands as bandlib
+            st["amax"] = torch.empty(1, dtype=torch.int32, device=dev)
+            st["bands"] = []
+            for k in range(self.nb):
+                r0, r1 = bandlib.band_rows(s.H, self.nb, k)
+                lo, hi, ht, hb = bandlib.band_input(s.H, r0, r1)
+                xv = st["x"][:, :, lo:hi]
+                st["bands"].append(dict(x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
+                                        x_scale=torch.empty(1, dtype=torch.float32, device=dev),
+                                        ht=ht, hb=hb, out=st["out"][:, :, r0:r1]))
+            del st["xq"]
+        return st
+
+    def launches_per_step(self):
+        return 1 + 2 * self.nb if self.nb else 3 * len(self.starts)
+
+    def _parts(self, st):
+        return st["chunks"] if self.chunk else [st]
+
+    def act(self, st):
+        q = self.qvae
+        if self.nb:
+            q.qvae_act_absmax(st["x"], st["amax"], self.stream)
+            for c in st["bands"]:
+                q.qvae_act_quant_from_absmax(c["x"], st["amax"], c["xq"], c["x_scale"], self.stream)
+            return
+        for c in self._parts(st):
+            q.qvae_act_absmax_quant(c["x"], c["xq"], c["x_scale"], c["ws"], self.stream)
+
+    def _conv_one(self, st, c):
+        q = self.qvae
+        if c.get("k", 0) == 0:
+            q.qvae_causal_conv3d_w8a8(c["xq"], c["x_scale"], st["packed"], self.s_w, self.b, c["out"], self.stream)
+        else:
+            q.qvae_causal_conv3d_w8a8_carry(c["xq"], c["x_scale"], st["packed"], self.s_w, self.b, c["out"],
+                                            self.stream)
+
+    def conv(self, st):
+        q = self.qvae
+        if self.nb:
+            for c in st["bands"]:
+                q.qvae_causal_conv3d_w8a8_band(c["xq"], c["ht"], c["hb"], c["x_scale"], st["packed"], self.s_w,
+                                               self.b, c["out"], self.stream)
+            return
+        for c in self._parts(st):
+            self._conv_one(st, c)
+
+    def step(self, st):
+        q = self.qvae
+        if self.nb:
+            q.qvae_act_absmax(st["x"], st["amax"], self.stream)
+            for c in st["bands"]:
+                q.qvae_act_quant_from_absmax(c["x"], st["amax"], c["xq"], c["x_scale"], self.stream)
+                q.qvae_causal_conv3d_w8a8_band(c["xq"], c["ht"], c["hb"], c["x_scale"], st["packed"], self.s_w,
+                                               self.b, c["out"], self.stream)
+            return
+        for c in self._parts(st):
+            q.qvae_act_absmax_quant(c["x"], c["xq"], c["x_scale"], c["ws"], self.stream)
+            self._conv_one(st, c)
+
 
 def run_ours(args):
     import math
@@ -276,138 +457,48 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    wl = synth.WORKLOADS[args.workload]
-    layer = synth.draw_workload(args.workload, seed=rank_seed(wl.seed, rank), only=[args.layer])[0]
-    s = layer.shape
-    w, b = layer.w.to(dev), layer.bias.to(dev)
-    packed0, s_w = qvae.quantize_weights(w)                # once, as at model load
-    torch.cuda.synchronize()
+    wl, idx = pick_layers(args)
+    layers = synth.draw_workload(args.workload, seed=rank_seed(wl.seed, rank), only=idx)
+    single = len(layers) == 1
+    if not single and (args.chunk or args.bands):
+        raise SystemExit("--chunk and --bands take one layer (--layer I)")
     # A side stream (CUDA graphs cannot capture the legacy default stream);
     # every launch and copy below runs on it.
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
+    jobs = [LayerJob(l, dev, stream, qvae, args, single) for l in layers]
+    torch.cuda.synchronize()
 
-    # Buffer sets (input, codes, output, packed weights) rotate so that every
-    # step reads and writes memory that is not in L2, as a decoder layer does:
-    # together the sets are more than three times the 126 MB L2.
-    per_set = x_bytes = layer.x.numel() * 2
-    per_set += layer.x.numel() + s.pixels * s.Cout * 2 + packed0.numel()
+    # Buffer sets (inputs, codes, outputs, packed weights of every layer) rotate
+    # so that every step reads and writes memory that is not in L2, as a
+    # decoder does: together the sets are more than three times the 126 MB L2.
+    per_set = sum(j.set_bytes() for j in jobs)
     n_sets = max(2, math.ceil(3 * L2_BYTES / per_set))
-    sets = []
-    for _ in range(n_sets):
-        sets.append(dict(
-            x=layer.x.to(dev), xq=torch.empty(layer.x.shape, dtype=torch.int8, device=dev),
-            x_scale=torch.empty(1, dtype=torch.float32, device=dev),
-            ws=torch.empty(qvae.qvae_act_workspace_bytes(layer.x.numel()), dtype=torch.uint8, device=dev),
-            out=torch.empty((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device=dev),
-            packed=packed0.clone()))
+    sets = [[j.make_set() for j in jobs] for _ in range(n_sets)]
 
-    # Streamed decode (--chunk C, one video): chunk k covers frames
-    # [kC, kC + C); its input is the view x[:, kC - 2 : kC + C] (the two frames
-    # before it carried), quantised as one tensor, then the carried-frame
-    # convolution; chunk 0 has no history and runs the causal convolution.
-    chunk = args.chunk if (args.chunk > 0 and s.T > args.chunk) else 0
-    if chunk and s.N != 1:
-        raise SystemExit("--chunk streams one video (N = 1)")
-    starts = list(range(0, s.T, chunk)) if chunk else [0]
-    if chunk:
-        for st in sets:
-            st["chunks"] = []
-            for k, t0 in enumerate(starts):
-                t1 = min(t0 + chunk, s.T)
-                xv = st["x"][:, (t0 - 2 if k else 0):t1]
-                st["chunks"].append(dict(
-                    k=k, x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
-                    x_scale=torch.empty(1, dtype=torch.float32, device=dev),
-                    ws=torch.empty(qvae.qvae_act_workspace_bytes(xv.numel()), dtype=torch.uint8, device=dev),
-                    out=st["out"][:, t0:t1]))
-            del st["xq"]
+    def step(ss):
+        for j, st in zip(jobs, ss):
+            j.step(st)
 
-    # Tiled decode (--bands B, one image): the whole image's absmax into a
-    # word, then per band its rows plus halo rows quantised from that word and
-    # the band convolution into the band's output rows.
-    nb = args.bands if args.bands > 1 else 0
-    if nb and s.N * s.T != 1:
-        raise SystemExit("--bands decodes one image (N = T = 1)")
-    if nb and chunk:
-        raise SystemExit("--bands and --chunk do not combine")
-    if nb:
-        from video_vae_decode_b200 import bands as bandlib
-        for st in sets:
-            st["amax"] = torch.empty(1, dtype=torch.int32, device=dev)
-            st["bands"] = []
-            for k in range(nb):
-                r0, r1 = bandlib.band_rows(s.H, nb, k)
-                lo, hi, ht, hb = bandlib.band_input(s.H, r0, r1)
-                xv = st["x"][:, :, lo:hi]
-                st["bands"].append(dict(x=xv, xq=torch.empty(xv.shape, dtype=torch.int8, device=dev),
-                                        x_scale=torch.empty(1, dtype=torch.float32, device=dev),
-                                        ht=ht, hb=hb, out=st["out"][:, :, r0:r1]))
-            del st["xq"]
-
-    def act_one(c):
-        qvae.qvae_act_absmax_quant(c["x"], c["xq"], c["x_scale"], c["ws"], stream)
-
-    def band_quant(st, c):
-        qvae.qvae_act_quant_from_absmax(c["x"], st["amax"], c["xq"], c["x_scale"], stream)
-
-    def band_conv(st, c):
-        qvae.qvae_causal_conv3d_w8a8_band(c["xq"], c["ht"], c["hb"], c["x_scale"], st["packed"], s_w, b,
-                                          c["out"], stream)
-
-    def conv_one(c, packed):
-        if c.get("k", 0) == 0:
-            qvae.qvae_causal_conv3d_w8a8(c["xq"], c["x_scale"], packed, s_w, b, c["out"], stream)
-        else:
-            qvae.qvae_causal_conv3d_w8a8_carry(c["xq"], c["x_scale"], packed, s_w, b, c["out"], stream)
-
-    def parts(st):
-        return st["chunks"] if chunk else [st]
-
-    def act(st):
-        if nb:
-            qvae.qvae_act_absmax(st["x"], st["amax"], stream)
-            for c in st["bands"]:
-                band_quant(st, c)
-            return
-        for c in parts(st):
-            act_one(c)
-
-    def conv(st):
-        if nb:
-            for c in st["bands"]:
-                band_conv(st, c)
-            return
-        for c in parts(st):
-            conv_one(c, st["packed"])
-
-    def step(st):
-        if nb:
-            qvae.qvae_act_absmax(st["x"], st["amax"], stream)
-            for c in st["bands"]:
-                band_quant(st, c)
-                band_conv(st, c)
-            return
-        for c in parts(st):
-            act_one(c)
-            conv_one(c, st["packed"])
-
-    # One CUDA graph per buffer set holds that set's step (the three kernels,
-    # with their programmatic launch dependencies): a replay costs the host one
-    # call, so the timed loop measures the device, not the Python launch path.
-    # First call of the layer in this process (tiling choice, tensor-map
+    # First call of the first layer in this process (tiling choice, tensor-map
     # encoding, kernel attributes and module load included), host wall clock.
     torch.cuda.synchronize()
     t_first = time.perf_counter()
-    step(sets[0])
+    jobs[0].step(sets[0][0])
     torch.cuda.synchronize()
     first_call_ms = (time.perf_counter() - t_first) * 1e3
+    for j, st in zip(jobs, sets[0]):
+        j.step(st)
+    torch.cuda.synchronize()
+    # One CUDA graph per buffer set holds that set's step (every layer's
+    # kernels, with their programmatic launch dependencies): a replay costs the
+    # host one call, so the timed loop measures the device.
     if args.launch == "graph":
         graphs = []
-        for st in sets:
+        for ss in sets:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                step(st)
+                step(ss)
             graphs.append(g)
         torch.cuda.synchronize()
 
@@ -442,51 +533,65 @@ def run_ours(args):
     if qvae.qvae_get_error() != 0:
         raise RuntimeError("device-side timeout during timing")
 
-    # ---- per-kernel durations (for the roofline): events around each launch.
-    # A GPU spin ahead of each group keeps the device behind the host, so the
-    # events time the kernels and not the host's launch gaps.
-    R = max(20, min(K, 400))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
-    for i in range(R):
-        st = sets[i % n_sets]
-        torch.cuda._sleep(SPIN_CYCLES)
-        ev[i][0].record(stream)
-        act(st)
-        ev[i][1].record(stream)
-        conv(st)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    act_ms = [a.elapsed_time(m) for a, m, _ in ev]
+    # ---- per-layer durations: events around each layer's activation passes,
+    # its convolution, and both back to back.  A GPU spin ahead of each group
+    # keeps the device behind the host, so the events time kernels and not
+    # the host's launch gaps.
+    R = max(10, min(K, 100 if single else 40))
+    per_layer = []
+    for li, j in enumerate(jobs):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(R)]
+        for i in range(R):
+            st = sets[i % n_sets][li]
+            torch.cuda._sleep(SPIN_CYCLES)
+            ev[i][0].record(stream)
+            j.act(st)
+            ev[i][1].record(stream)
+            j.conv(st)
+            ev[i][2].record(stream)
+            torch.cuda._sleep(SPIN_CYCLES)
+            ev2[i][0].record(stream)
+            j.step(st)
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize()
+        act_ms = [a.elapsed_time(m) for a, m, _ in ev]
+        conv_ms = [m.elapsed_time(z) for _, m, z in ev]
+        layer_ms = [a.elapsed_time(z) for a, z in ev2]
+        per_layer.append(dict(act=statistics.mean(act_ms), conv=statistics.mean(conv_ms),
+                              conv_median=statistics.median(conv_ms), layer=statistics.mean(layer_ms)))
+    conv_launches = R
 
-    # A resolution switch: the first call of the same layer at the spatial size
+    # A resolution switch: the first call of the first layer at the spatial size
     # scaled by 840/1024 (the pages' switch from 1024x1024 to 840x1256 output),
     # in this warm process; nothing is compiled per shape.
-    Hs, Ws = max(1, (s.H * 840) // 1024), max(1, (s.W * 1256) // 1024)
-    xs = torch.randn((s.N, s.T, Hs, Ws, s.Cin), device=dev).to(torch.bfloat16)
+    s0 = jobs[0].s
+    Hs, Ws = max(1, (s0.H * 840) // 1024), max(1, (s0.W * 1256) // 1024)
+    xs = torch.randn((s0.N, s0.T, Hs, Ws, s0.Cin), device=dev).to(torch.bfloat16)
     xqs = torch.empty(xs.shape, dtype=torch.int8, device=dev)
     scs = torch.empty(1, dtype=torch.float32, device=dev)
     wss = torch.empty(qvae.qvae_act_workspace_bytes(xs.numel()), dtype=torch.uint8, device=dev)
-    outs = torch.empty((s.N, s.T, Hs, Ws, s.Cout), dtype=torch.bfloat16, device=dev)
+    outs = torch.empty((s0.N, s0.T, Hs, Ws, s0.Cout), dtype=torch.bfloat16, device=dev)
     switch_ms = []
     for _ in range(2):                            # first call, then the same call warm
         torch.cuda.synchronize()
         t_sw = time.perf_counter()
         qvae.qvae_act_absmax_quant(xs, xqs, scs, wss, stream)
-        qvae.qvae_causal_conv3d_w8a8(xqs, scs, packed0, s_w, b, outs, stream)
+        qvae.qvae_causal_conv3d_w8a8(xqs, scs, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, stream)
         torch.cuda.synchronize()
         switch_ms.append((time.perf_counter() - t_sw) * 1e3)
     del xs, xqs, wss, outs
-    conv_ms = [m.elapsed_time(z) for _, m, z in ev]
 
-    # ---- end to end: pinned host input -> device -> layer -> pinned host output.
-    # Every step copies its own input in and its own output back; as in a
+    # ---- end to end: pinned host inputs -> device -> layers -> pinned host outputs.
+    # Every step copies its own inputs in and its own outputs back; as in a
     # serving loop, the copies run on their own streams (one per direction)
-    # and overlap the neighbouring steps' compute: step i + 1's input lands
-    # in its buffer set while step i computes and step i - 1's output leaves.
-    x_host = layer.x.pin_memory()
-    out_hosts = [torch.empty(sets[0]["out"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    # and overlap the neighbouring steps' compute: step i + 1's inputs land
+    # in its buffer set while step i computes and step i - 1's outputs leave.
+    x_hosts = [j.layer.x.pin_memory() for j in jobs]
+    out_hosts = [[torch.empty(sets[0][li]["out"].shape, dtype=torch.bfloat16).pin_memory()
+                  for li in range(len(jobs))] for _ in range(2)]
     h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    e2e_steps = max(3, min(K, 200))
+    e2e_steps = max(3, min(K, 200 if single else 12))
     loaded = [torch.cuda.Event() for _ in range(n_sets)]
     computed = [torch.cuda.Event() for _ in range(n_sets)]
     drained = [torch.cuda.Event() for _ in range(n_sets)]
@@ -497,25 +602,31 @@ def run_ours(args):
     e2e_a.record(h2d_stream)
     for i in range(e2e_steps):
         k = i % n_sets
-        st = sets[k]
-        h2d_stream.wait_event(drained[k])           # the set's previous output has left the device
+        ss = sets[k]
+        h2d_stream.wait_event(drained[k])           # the set's previous outputs have left the device
         with torch.cuda.stream(h2d_stream):
-            st["x"].copy_(x_host, non_blocking=True)
+            for st, xh in zip(ss, x_hosts):
+                st["x"].copy_(xh, non_blocking=True)
         loaded[k].record(h2d_stream)
         stream.wait_event(loaded[k])
-        act(st)
-        conv(st)
+        for j, st in zip(jobs, ss):
+            j.act(st)
+            j.conv(st)
         computed[k].record(stream)
         d2h_stream.wait_event(computed[k])
         with torch.cuda.stream(d2h_stream):
-            out_hosts[i % 2].copy_(st["out"], non_blocking=True)
+            for st, oh in zip(ss, out_hosts[i % 2]):
+                oh.copy_(st["out"], non_blocking=True)
         drained[k].record(d2h_stream)
     e2e_b.record(d2h_stream)
     torch.cuda.synchronize()
     e2e_ms = e2e_a.elapsed_time(e2e_b) / e2e_steps
 
-    ops = s.ops()
-    total_ms_max, e2e_ms_max, conv_ms_max = max_over_ranks([total_ms, e2e_ms, statistics.mean(conv_ms)], dev)
+    int8_tops = int8_cublas_tops(dev) if rank == 0 else None
+
+    ops = sum(j.s.ops() for j in jobs)
+    conv_total = sum(p["conv"] for p in per_layer)
+    total_ms_max, e2e_ms_max, conv_total_max = max_over_ranks([total_ms, e2e_ms, conv_total], dev)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -525,50 +636,132 @@ def run_ours(args):
     value = ops * world / (ms_per_step * 1e-3) / 1e12
     bf16_burst, bf16_sust, peak_src = measured_peaks()
     peak = bf16_burst * INT8_PER_BF16
-    conv_mean = statistics.mean(conv_ms)
-    conv_tops = ops / (conv_mean * 1e-3) / 1e12
-    traffic = profiled_traffic(args.workload)
+    conv_tops = ops / (conv_total_max * 1e-3) / 1e12
+    layer_entries = []
+    traffic = []
+    for li, (j, p) in enumerate(zip(jobs, per_layer)):
+        lops = j.s.ops()
+        key = args.workload if single and len(wl.layers) == 1 else f"{args.workload}[{idx[li]}]"
+        tr = profiled_traffic(key)
+        traffic.append(tr)
+        numel = j.layer.x.numel()
+        layer_entries.append({
+            "layer": layer_name(j.layer), "index": idx[li], "ops": lops,
+            "ms": p["layer"], "act_ms": p["act"], "conv_ms": p["conv"], "conv_ms_median": p["conv_median"],
+            "layer_tops": lops / (p["layer"] * 1e-3) / 1e12, "conv_tops": lops / (p["conv"] * 1e-3) / 1e12,
+            "conv_frac": lops / (p["conv"] * 1e-3) / 1e12 / peak,
+            "act_gbs_moved_5B": 5 * numel / (p["act"] * 1e-3) / 1e9,
+            "tiling": qvae.qvae_get_conv_tiling(j.s.N, j.s.T, j.s.H, j.s.W, j.s.Cin, j.s.Cout),
+            "dram_bytes_per_conv_launch": tr})
+    traffic_mean = (sum(traffic) / len(traffic)) if all(t is not None for t in traffic) else None
+    h2d = sum(j.layer.x.numel() * 2 for j in jobs)
+    d2h = sum(j.s.pixels * j.s.Cout * 2 for j in jobs)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
-        "config": {"workload": args.workload, "layer": layer_name(layer), "arithmetic": ARITHMETIC,
-                   "tiling": qvae.qvae_get_conv_tiling(s.N, s.T, s.H, s.W, s.Cin, s.Cout),
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": DATA,
+        "config": {"workload": args.workload, "layers": [layer_name(j.layer) for j in jobs],
+                   "arithmetic": ARITHMETIC,
                    "l2": (f"inputs, codes, outputs and packed weights rotate over {n_sets} buffer sets "
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
-                   "launch": ("one CUDA graph replay per step (act absmax, act quantise, conv)"
+                   "launch": ("one CUDA graph replay per step (per layer: act absmax, act quantise, conv)"
                               if args.launch == "graph" else "direct launches from Python"),
-                   "ops_per_layer": ops,
-                   "stream_chunk": (f"{chunk} frames, two carried" if chunk else None),
-                   "row_bands": nb or None},
-        "ms_per_layer": {"step": ms_per_step, "act_absmax_quant": statistics.mean(act_ms),
-                         "conv": conv_mean, "conv_median": statistics.median(conv_ms)},
+                   "ops_per_step": ops,
+                   "stream_chunk": (f"{jobs[0].chunk} frames, two carried" if jobs[0].chunk else None),
+                   "row_bands": jobs[0].nb or None},
+        "ms_per_layer": {e["layer"]: e["ms"] for e in layer_entries},
+        "per_layer": layer_entries,
         "conv_tops": conv_tops,
-        "act_gbs": {"moved_5B": 5 * layer.x.numel() / (statistics.mean(act_ms) * 1e-3) / 1e9,
-                    "algorithmic_3B": 3 * layer.x.numel() / (statistics.mean(act_ms) * 1e-3) / 1e9,
-                    "note": "activation passes: 5 B per element moved (bf16 read twice, int8 written; "
-                            "the second read hits L2 when x fits), 3 B algorithmic; measured copy "
-                            "bandwidth 6557 GB/s"},
-        "first_call_ms": {"process_first": first_call_ms,
-                          "resolution_switch": {"shape": f"{Hs}x{Ws}", "first": switch_ms[0],
-                                                "warm": switch_ms[1]},
-                          "note": "host wall clock, act + conv with a device synchronise"},
         "pct_datasheet_int8_peak": 100.0 * conv_tops / DATASHEET_INT8_TOPS,
+        "first_call_ms": {"process_first": first_call_ms,
+                          "resolution_switch": {"shape": f"{Hs}x{Ws}", "first": switch_ms[0], "warm": switch_ms[1]},
+                          "note": "host wall clock, act + conv of the first layer with a device synchronise"},
         "roofline": {"bound": "tensor", "achieved": conv_tops, "peak": peak, "unit": "TOPS",
-                     "frac": conv_tops / peak, "traffic": traffic,
+                     "frac": conv_tops / peak, "traffic": traffic_mean,
                      "peak_source": f"{peak_src} bf16 burst {bf16_burst} TFLOP/s x {INT8_PER_BF16} "
                                     "(nominal dense INT8/BF16 ratio)",
-                     "kernel": "conv3d_w8a8_kernel", "kernel_ms_mean": conv_mean, "launches": R},
+                     "int8_cublas_tops": int8_tops,
+                     "frac_of_int8_cublas": (conv_tops / int8_tops) if int8_tops else None,
+                     "kernel": "conv3d_w8a8_kernel",
+                     "kernel_ms_mean": conv_total_max / len(jobs), "launches": conv_launches * len(jobs),
+                     "note": ("achieved = the layers' ops over the sum of their convolutions' mean CUDA-event "
+                              "times; traffic = mean DRAM bytes per conv launch over the layers")},
         "e2e": {"value": ops * world / (e2e_ms_max * 1e-3) / 1e12, "unit": UNIT,
-                "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": s.pixels * s.Cout * 2},
-        "gpu_launches": K * (1 + 2 * nb if nb else 3 * len(starts)),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * sum(j.launches_per_step() for j in jobs),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
-        cb = oracle_baseline(layer, args.cpu_seconds)
+        cb = oracle_baseline([j.layer for j in jobs], args.cpu_seconds)
         cb.pop("seconds", None)
         line["cpu_baseline"] = cb
+    print(json.dumps(line))
+    return 0
+
+
+def run_split(args):
+    """One image layer split across the ranks by row bands (bands.decode_split):
+    per step, the local absmax, an all-reduce MAX of one 4-byte word, one halo
+    row to and from each neighbour, then this rank's band quantisation and band
+    convolution.  Strong scaling: every step decodes the same one image."""
+    import torch
+    import torch.distributed as dist
+    from video_vae_decode_b200 import bands, qvae, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wl = synth.WORKLOADS[args.workload]
+    li = args.layer if args.layer >= 0 else len(wl.layers) - 1
+    layer = synth.draw_workload(args.workload, only=[li])[0]      # the same image on every rank
+    s = layer.shape
+    if s.N * s.T != 1:
+        raise SystemExit("--split decodes one image (N = T = 1)")
+    r0, r1 = bands.band_rows(s.H, world, rank)
+    x_rows = layer.x[:, :, r0:r1].contiguous().to(dev)
+    packed, s_w = qvae.quantize_weights(layer.w.to(dev))
+    ops_ = bands.QvaeBandOps(packed, s_w, layer.bias.to(dev), s.Cout)
+    out = torch.empty((1, 1, r1 - r0, s.W, s.Cout), dtype=torch.bfloat16, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        bands.decode_split(x_rows, ops_, rank, world, s.Cout, out=out)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            bands.decode_split(x_rows, ops_, rank, world, s.Cout, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if qvae.qvae_get_error() != 0:
+        raise RuntimeError("device-side timeout")
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    ops = s.ops()
+    line = {
+        "metric": METRIC + ", one image split across GPUs by row bands", "value": ops / (ms * 1e-3) / 1e12,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "int8", "data": DATA,
+        "config": {"workload": args.workload, "layer": layer_name(layer), "arithmetic": ARITHMETIC,
+                   "split": f"{world} row bands; all-reduce MAX of the activation maximum, one halo row per "
+                            "neighbour (NCCL point-to-point), band quantise + band conv",
+                   "launch": "direct launches from Python (NCCL calls between the kernels)"},
+        "gpu_launches": args.steps * 3,
+        "clocks": clk.summary(),
+    }
     print(json.dumps(line))
     return 0
 
@@ -650,8 +843,7 @@ def run_chain(args):
     line = {
         "metric": METRIC + ", layer chain", "value": ops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded stand-in for the decoder's latents and random-init weights)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": DATA,
         "config": {"workload": args.workload, "chain": [layer_name(t) for t in tens], "arithmetic": ARITHMETIC,
                    "l2": f"{n_sets} buffer sets rotate ({n_sets * per_set / 2**20:.0f} MiB)",
                    "launch": "one CUDA graph replay per chain (qvae_decode_layers)", "ops": ops},
@@ -669,6 +861,8 @@ def main():
         return run_reference(args)
     if args.chain:
         return run_chain(args)
+    if args.split:
+        return run_split(args)
     return run_ours(args)
 
 

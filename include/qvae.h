@@ -234,12 +234,57 @@ int qvae_causal_conv3d_w8a8_band_acc32(const qvae_shape* shape, int32_t halo_top
                                        const int8_t* xq_band, const int8_t* wq_packed, int32_t* acc,
                                        void* stream);
 
+/* ------------------------------------------------- native-precision layer -- */
+
+/* Bytes of a native layer's packed bf16 weights:
+ * 27 taps x ceil(Cin/64) chunks x Cout rows x 128 bytes. */
+size_t qvae_packed_weight_bytes_bf16(int32_t Cin, int32_t Cout);
+
+/*
+ * One-time repack of a native-precision layer's weights (no quantisation).
+ * The release note's Aggressive preset keeps two decoder convolutions in
+ * their original precision (its exclusion rule names
+ * decoder.upsamples.14.residual.2 and .residual.6); they run on the same
+ * tiled convolution with bf16 operands.
+ *   w_bf16    [Cout][Cin][3][3][3] bf16, the PyTorch Conv3d weight layout.
+ *   w_packed  qvae_packed_weight_bytes_bf16(Cin, Cout) bytes, written:
+ *             [tap][chunk][Cout][64] bf16, tap = (kt*3 + kh)*3 + kw, each
+ *             128-byte row holding 64 input channels in the 128-byte swizzle
+ *             (16-byte group g at position g ^ (co % 8)), zeros beyond Cin.
+ * Needs Cin % 32 == 0 and Cout % 32 == 0.  Ends with an empty kernel, like
+ * qvae_quantize_weights (see the ordering note of qvae_causal_conv3d_w8a8).
+ */
+int qvae_pack_weights_bf16(int32_t Cin, int32_t Cout, const void* w_bf16, void* w_packed, void* stream);
+
+/*
+ * The causal 3x3x3 convolution in native precision:
+ *   out[n,t,h,w,co] = bf16_rne( acc + bias[co] ),
+ *   acc = sum over kt,kh,kw,ci of x[n, t+kt-2, h+kh-1, w+kw-1, ci] * w[co, ci, kt, kh, kw]
+ * evaluated on the tensor cores (kind::f16) with bf16 products accumulated
+ * in fp32 (zero outside the tensor, as for the W8A8 layer).  The sum is not
+ * exact: it differs from the exact value by the fp32 rounding of its
+ * accumulation, at most 2^-12 of the sum of |x * w| over the layer's shapes.
+ *   x_bf16    [N][T][H][W][Cin] bf16.   w_packed from qvae_pack_weights_bf16.
+ *   bias_bf16 [Cout] bf16 or NULL.      out_bf16 [N][T][H][W][Cout] bf16.
+ * Errors and ordering as qvae_causal_conv3d_w8a8.
+ */
+int qvae_causal_conv3d_bf16(const qvae_shape* shape, const void* x_bf16, const void* w_packed,
+                            const void* bias_bf16, void* out_bf16, void* stream);
+
+/* The native-precision convolution writing its raw fp32 sums acc [N][T][H][W][Cout]
+ * (no bias) instead of the bf16 output. */
+int qvae_causal_conv3d_bf16_acc32(const qvae_shape* shape, const void* x_bf16, const void* w_packed,
+                                  float* acc, void* stream);
+
 /* ---------------------------------------------------------- layer chain -- */
 
 /*
  * One decoder layer for qvae_decode_layers.  quantized == 0 marks a layer
  * kept in native precision (the release note's Aggressive preset keeps 2 of
- * 28); the library skips it and the caller runs it.
+ * 28): with wq_packed holding its bf16 weights packed by
+ * qvae_pack_weights_bf16 the library runs it with qvae_causal_conv3d_bf16
+ * (w_scale unused); with wq_packed == NULL the library skips it and the
+ * caller runs it.
  */
 typedef struct qvae_layer {
   qvae_shape shape;
@@ -247,8 +292,8 @@ typedef struct qvae_layer {
   int32_t reserved;          /* set to 0 */
   const void* x;             /* bf16 [N][T][H][W][Cin] */
   void* out;                 /* bf16 [N][T][H][W][Cout] */
-  const int8_t* wq_packed;   /* from qvae_quantize_weights */
-  const float* w_scale;      /* [Cout] */
+  const void* wq_packed;     /* qvae_quantize_weights (quantized), qvae_pack_weights_bf16 (native) or NULL */
+  const float* w_scale;      /* [Cout] (quantized layers) */
   const void* bias;          /* bf16 [Cout] or NULL */
 } qvae_layer;
 
@@ -256,13 +301,15 @@ typedef struct qvae_layer {
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
 
 /*
- * For each layer with quantized != 0, in order on one stream: activation
- * absmax + quantise into the workspace, then the convolution into `out`.
- * All layers are validated before anything is launched.  When a quantised
- * layer's `out` is the next quantised layer's `x` (same N, T, H, W and
- * Cout == next Cin), the convolution also accumulates the maximum bf16
- * magnitude it writes into the workspace and the next layer skips its absmax
- * pass: codes, scales and outputs are the same as layer-by-layer calls.
+ * In order on one stream, for each quantised layer: activation absmax +
+ * quantise into the workspace, then the W8A8 convolution into `out`; for each
+ * native layer with packed bf16 weights: the bf16 convolution into `out`;
+ * native layers without weights are skipped.  All layers are validated
+ * before anything is launched.  When a layer's `out` is the next layer's `x`
+ * and the next layer is quantised (same N, T, H, W and Cout == next Cin), the
+ * convolution also accumulates the maximum bf16 magnitude it writes into the
+ * workspace and the next layer skips its absmax pass: codes, scales and
+ * outputs are the same as layer-by-layer calls.
  */
 int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
                        size_t workspace_bytes, void* stream);

@@ -87,7 +87,13 @@ def test_decode_layers_validates_everything_first():
     arr[1].shape = qvae.make_shape(1, 1, 8, 8, 48, 64)
     need = L.qvae_decode_workspace_bytes(arr, 2)
     assert L.qvae_decode_layers(arr, 2, FAKE, need, None) == qvae.QVAE_ERR_SHAPE
-    arr[1].quantized = 0                                   # pass-through layers are not checked
+    arr[1].quantized = 0                                   # a native layer with weights is run: checked
+    assert L.qvae_decode_layers(arr, 2, FAKE, need, None) == qvae.QVAE_ERR_SHAPE
+    arr[1].shape = qvae.make_shape(1, 1, 8, 8, 64, 64)
+    arr[1].x = 0x10008
+    assert L.qvae_decode_layers(arr, 2, FAKE, need, None) == qvae.QVAE_ERR_ALIGN
+    arr[1].shape = qvae.make_shape(1, 1, 8, 8, 48, 64)
+    arr[1].wq_packed = None                                # without weights it is skipped: not checked
     need = L.qvae_decode_workspace_bytes(arr, 2)
     assert need >= 8 * 8 * 64
     assert L.qvae_decode_layers(arr, 2, FAKE, need - 1, None) == qvae.QVAE_ERR_ARG
@@ -175,3 +181,24 @@ def test_stream_band_and_split_activation_argument_checks():
     assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
     assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, None, FAKE, None) == qvae.QVAE_ERR_ARG
     assert L.qvae_act_quant_from_absmax(FAKE, 100, FAKE, FAKE_ODD, FAKE, None) == qvae.QVAE_ERR_ALIGN
+
+
+def test_native_layer_argument_checks():
+    L = qvae.lib()
+    assert qvae.qvae_packed_weight_bytes_bf16(96, 96) == 27 * 2 * 96 * 128
+    assert qvae.qvae_packed_weight_bytes_bf16(384, 192) == 27 * 6 * 192 * 128
+    assert qvae.qvae_packed_weight_bytes_bf16(32, 32) == 27 * 1 * 32 * 128
+    assert qvae.qvae_packed_weight_bytes_bf16(0, 32) == 0
+    assert L.qvae_pack_weights_bf16(48, 64, FAKE, FAKE, None) == qvae.QVAE_ERR_SHAPE
+    assert L.qvae_pack_weights_bf16(64, 64, None, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert L.qvae_pack_weights_bf16(64, 64, FAKE, FAKE_ODD, None) == qvae.QVAE_ERR_ALIGN
+    ok = qvae.make_shape(1, 1, 8, 8, 64, 64)
+    conv = L.qvae_causal_conv3d_bf16
+    assert conv(ctypes.byref(qvae.make_shape(1, 1, 8, 8, 48, 64)), FAKE, FAKE, None, FAKE, None) == qvae.QVAE_ERR_SHAPE
+    assert conv(ctypes.byref(ok), None, FAKE, None, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert conv(ctypes.byref(ok), FAKE, None, None, FAKE, None) == qvae.QVAE_ERR_ARG
+    assert conv(ctypes.byref(ok), FAKE, FAKE, None, None, None) == qvae.QVAE_ERR_ARG
+    assert conv(ctypes.byref(ok), FAKE_ODD, FAKE, None, FAKE, None) == qvae.QVAE_ERR_ALIGN
+    assert conv(ctypes.byref(ok), FAKE, FAKE, None, FAKE_ODD, None) == qvae.QVAE_ERR_ALIGN
+    assert conv(ctypes.byref(qvae.make_shape(1, 1, 0, 8, 64, 64)), None, None, None, None, None) == qvae.QVAE_OK
+    assert L.qvae_causal_conv3d_bf16_acc32(ctypes.byref(ok), FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG

@@ -110,8 +110,10 @@ def _chain(q, shapes, passthrough=(), seed=31):
         w, b = t.w.cuda(), t.bias.cuda()
         packed, s_w = q.quantize_weights(w)
         out = torch.zeros((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device="cuda")
-        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=i not in passthrough,
-                          w=w))
+        quantized = i not in passthrough
+        # a pass-through layer without weights is skipped by the library (the caller runs it)
+        specs.append(dict(x=x, out=out, wq_packed=packed if quantized else None, w_scale=s_w, bias=b,
+                          quantized=quantized, w=w))
         weights.append((packed, s_w, b, s.Cout))
         x = out
     return specs, weights

@@ -334,7 +334,9 @@ def test_decode_layers_matches_single_calls_and_skips_passthrough(q):
         x, w, b = t.x.cuda(), t.w.cuda(), t.bias.cuda()
         packed, s_w = q.quantize_weights(w)
         out = torch.full((s.N, s.T, s.H, s.W, s.Cout), 7.0, dtype=torch.bfloat16, device="cuda")
-        specs.append(dict(x=x, out=out, wq_packed=packed, w_scale=s_w, bias=b, quantized=(i != 1)))
+        # layer 1 is a native layer without weights: the library skips it
+        specs.append(dict(x=x, out=out, wq_packed=None if i == 1 else packed, w_scale=s_w, bias=b,
+                          quantized=(i != 1)))
         xq, s_a = q.act_absmax_quant(x)
         refs.append(q.causal_conv3d_w8a8(xq, s_a, packed, s_w, b, s.Cout))
     layers = q.make_layers(specs)

@@ -112,7 +112,8 @@ def decode_split(x_rows: torch.Tensor, ops, rank: int, world: int, Cout: int, gr
     activation scale) and one row to and from each neighbour.
     """
     amax = ops.absmax(x_rows)
-    dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    if world > 1:
+        dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
     x_band, ht, hb = exchange_halo_rows(x_rows, rank, world, group)
     xq, scale = ops.quant(x_band, amax)
     if out is None:

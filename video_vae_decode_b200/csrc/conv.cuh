@@ -54,6 +54,14 @@
 // whose input holds halo rows in place of the top / bottom padding
 // (halo_top), raw INT32 accumulators instead of the bf16 output (kAcc32), and
 // the maximum |output| accumulated for the next layer's quantiser (out_amax).
+//
+// Native precision (conv3d_bf16_kernel).  The release note's Aggressive
+// preset keeps two decoder convolutions in their original precision.  They
+// run on the same body with bf16 operands: a 128-byte shared-memory line then
+// holds 64 channels instead of 128 codes and one tcgen05.mma.kind::f16 step
+// consumes K = 16 bf16 values (32 bytes) instead of 32 codes, so the boxes,
+// rings, tap offsets and descriptors are unchanged; the accumulators are fp32
+// and the epilogue computes bf16_rne(acc + bias).
 #pragma once
 
 #include <cuda.h>
@@ -75,7 +83,8 @@ struct ConvArgs {
   int N, T, H, W, Cin, Cout;
   int MS, NT;                 // sub-tiles per CTA tile, output channels per CTA tile
   int tiles_w, tiles_h, tiles_n, num_tiles;  // tiles_h counts CTA-pair row bands in pair mode
-  int nchunks, last_ksteps;   // 128-channel chunks; 32-channel k-steps in the last one
+  int nchunks, last_ksteps;   // 128-byte channel chunks; 32-byte k-steps in the last one
+  int chunk_elems;            // channels per 128-byte chunk: 128 (int8 codes) or 64 (bf16 values)
   int SA, SB, acc_stages;     // pipeline depths
   int G;                      // taps per weight stage (1 or 3; 9 / G stages per 128-channel chunk)
   int split;                  // per-sub-tile accumulator hand-off (one accumulator buffer, MS >= 2, SB >= 9 / G)
@@ -147,11 +156,11 @@ struct MmaRings {
 // starts) while the later sub-tiles still run, and sub-tile s of the next
 // tile starts as soon as its epilogue has released it.  Returns false when a
 // wait gave up (abort or time limit).
-template <bool kPair, int kMS, int kG>
+template <bool kBf16, bool kPair, int kMS, int kG>
 __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
                                                volatile int* abort_flag, uint64_t limit, int first_tile,
                                                int tile_step, uint32_t rank, bool& issued) {
-  const uint32_t idesc = idesc_i8(kPair ? 256 : 128, a.NT);
+  const uint32_t idesc = kBf16 ? idesc_bf16(kPair ? 256 : 128, a.NT) : idesc_i8(kPair ? 256 : 128, a.NT);
   const uint64_t a_desc0 = sw128_kmajor_desc(r.a_ring, kGroupStride);
   const uint64_t b_desc0 = sw128_kmajor_desc(r.b_ring, 1024u);
   const uint32_t a_stage16 = a.a_stage_bytes >> 4, b_stage16 = a.b_stage_bytes >> 4;
@@ -164,7 +173,13 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
   bool b_ready = false;  // b_full of stage bs already seen complete
   auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
-    if (kPair) {
+    if (kBf16) {
+      if (kPair) {
+        mma_bf16_pair(d, ad, bd, idesc, acc);
+      } else {
+        mma_bf16(d, ad, bd, idesc, acc);
+      }
+    } else if (kPair) {
       mma_i8_pair(d, ad, bd, idesc, acc);
     } else {
       mma_i8(d, ad, bd, idesc, acc);
@@ -295,10 +310,15 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   return true;
 }
 
-template <bool kAcc32, bool kPair>
-__global__ void __launch_bounds__(kConvThreads, 1)
-    conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                       const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
+// The body of both convolution kernels.  kBf16: the operands are bf16 values
+// (kind::f16, fp32 accumulators, output bf16(acc + bias)); otherwise INT8
+// codes (kind::i8, INT32 accumulators, output bf16(acc * scale + bias)).  In
+// shared memory both are 128-byte lines per pixel -- 128 codes or 64 bf16
+// channels -- and one MMA step consumes 32 bytes of K, so the tiling, the
+// rings and the tap offsets are the same.
+template <bool kBf16, bool kAcc32, bool kPair>
+__device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w,
+                                            const CUtensorMap& tmap_out, const ConvArgs& a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -411,11 +431,11 @@ __global__ void __launch_bounds__(kConvThreads, 1)
           const uint32_t bar = a_full + 8 * as;
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
           if (kPair) {
-            tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * 128, c.w0 - 1,
-                             c.h0 - 1 + a.halo_top, frame, c.n);
+            tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * a.chunk_elems,
+                             c.w0 - 1, c.h0 - 1 + a.halo_top, frame, c.n);
           } else {
-            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * 128, c.w0 - 1, c.h0 - 1 + a.halo_top, frame,
-                        c.n);
+            tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * a.chunk_elems, c.w0 - 1,
+                        c.h0 - 1 + a.halo_top, frame, c.n);
           }
         }
         a_armed |= 1u << as;
@@ -443,8 +463,9 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     bool issued = false;
     bool ok;
     auto run = [&](auto ms, auto g) {
-      return mma_issue_loop<kPair, decltype(ms)::value, decltype(g)::value>(a, r, abort_flag, limit, first_tile,
-                                                                           tile_step, rank, issued);
+      return mma_issue_loop<kBf16, kPair, decltype(ms)::value, decltype(g)::value>(a, r, abort_flag, limit,
+                                                                                  first_tile, tile_step, rank,
+                                                                                  issued);
     };
     using G1 = std::integral_constant<int, 1>;
     using G3 = std::integral_constant<int, 3>;
@@ -507,9 +528,9 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     // lets the previous tile's slices finish reading the old table.
     auto fill_table = [&](int co0) {
       named_barrier_sync(1, 32 * kEpiWarps);
-      const float sa = *a.x_scale;
+      const float sa = kBf16 ? 1.0f : *a.x_scale;
       for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
-        sc[j] = __fmul_rn(sa, a.w_scale[co0 + j]);
+        sc[j] = kBf16 ? 1.0f : __fmul_rn(sa, a.w_scale[co0 + j]);
         bi[j] = a.bias ? __bfloat162float(a.bias[co0 + j]) : 0.0f;
       }
       scale_co0 = co0;
@@ -554,12 +575,20 @@ __global__ void __launch_bounds__(kConvThreads, 1)
               // y = float(acc) * scale, rounded, then + bias, rounded.  The
               // scalar _rn intrinsics are never contracted into an FMA (packed
               // f32x2 multiply + add were: one rounding instead of two).
-              const float4 f = sc4[e];
               const float4 b = bi4[e];
-              const float y0 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e])), f.x), b.x);
-              const float y1 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 1])), f.y), b.y);
-              const float y2 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 2])), f.z), b.z);
-              const float y3 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 3])), f.w), b.w);
+              float y0, y1, y2, y3;
+              if (kBf16) {  // fp32 accumulators: y = acc + bias
+                y0 = __fadd_rn(__uint_as_float(v[4 * e]), b.x);
+                y1 = __fadd_rn(__uint_as_float(v[4 * e + 1]), b.y);
+                y2 = __fadd_rn(__uint_as_float(v[4 * e + 2]), b.z);
+                y3 = __fadd_rn(__uint_as_float(v[4 * e + 3]), b.w);
+              } else {
+                const float4 f = sc4[e];
+                y0 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e])), f.x), b.x);
+                y1 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 1])), f.y), b.y);
+                y2 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 2])), f.z), b.z);
+                y3 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 3])), f.w), b.w);
+              }
               const __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
               const __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
               packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
@@ -655,6 +684,22 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       tmem_dealloc(tmem_base, a.tmem_cols);
     }
   }
+}
+
+// W8A8 convolution: INT8 codes, INT32 accumulators, FP32 rescale + bias.
+template <bool kAcc32, bool kPair>
+__global__ void __launch_bounds__(kConvThreads, 1)
+    conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
+  conv3d_body<false, kAcc32, kPair>(tmap_x, tmap_w, tmap_out, a);
+}
+
+// Native-precision convolution: bf16 values, fp32 accumulators, + bias.
+template <bool kAcc32, bool kPair>
+__global__ void __launch_bounds__(kConvThreads, 1)
+    conv3d_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
+  conv3d_body<true, kAcc32, kPair>(tmap_x, tmap_w, tmap_out, a);
 }
 
 // A wait that nothing satisfies: checks that a bounded wait gives up, raises

@@ -269,4 +269,31 @@ __global__ void weight_pack_kernel(const uint16_t* __restrict__ w, int Cin, int 
   }
 }
 
+// bf16 weights of a native-precision layer in the convolution's consumption
+// order (no quantisation).  One thread per packed bf16 value:
+//   packed[tap][chunk][co][64]   tap = (kt * 3 + kh) * 3 + kw, chunk = 64 input channels (128 bytes);
+// inside a 128-byte row the 16-byte group g holds channels chunk*64 + (g ^ (co & 7))*8 + [0,8)
+// (the same 128-byte swizzle as the INT8 packing); channels beyond Cin are zero.
+__global__ void weight_pack_bf16_kernel(const uint16_t* __restrict__ w, int Cin, int Cout, int nchunks,
+                                        uint16_t* __restrict__ packed) {
+  const int64_t total = static_cast<int64_t>(27) * nchunks * Cout * 64;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(idx & 63);  // bf16 slot in the 128-byte row
+    int64_t rest = idx >> 6;
+    const int co = static_cast<int>(rest % Cout);
+    rest /= Cout;
+    const int chunk = static_cast<int>(rest % nchunks);
+    const int tap = static_cast<int>(rest / nchunks);
+    const int g = (e >> 3) ^ (co & 7);
+    const int ci = chunk * 64 + g * 8 + (e & 7);
+    uint16_t v = 0;
+    if (ci < Cin) {
+      const int kt = tap / 9, kh = (tap / 3) % 3, kw = tap % 3;
+      v = w[((static_cast<int64_t>(co) * Cin + ci) * 3 + kt) * 9 + kh * 3 + kw];
+    }
+    packed[idx] = v;
+  }
+}
+
 }  // namespace qvae

@@ -34,7 +34,7 @@ std::atomic<int32_t> g_cta_limit{0};    // cap on the conv grid (0 = one CTA per
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
-bool g_conv_attr_set[kMaxDevices][4] = {};
+bool g_conv_attr_set[kMaxDevices][8] = {};
 int g_max_clusters[kMaxDevices] = {0};
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
@@ -284,21 +284,25 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
 // the previous chunk of a streamed video (output frames are the last T).
 // halo_top / halo_bot: xq holds H + halo_top + halo_bot rows, output row h
 // reading input rows h + halo_top - 1 .. h + halo_top + 1 (a row band).
-int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
-                const int8_t* wq, const float* w_scale, const void* bias, void* out, int32_t* acc,
+// bf16: the native-precision convolution -- xq holds bf16 values, wq the bf16
+// packing, acc (accumulator mode) receives fp32 sums; no scales.  It is tiled
+// as the INT8 convolution of twice the channels (the same bytes per pixel).
+int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
+                const void* wq, const float* w_scale, const void* bias, void* out, void* acc,
                 cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr, int halo_top = 0,
-                int halo_bot = 0) {
+                int halo_bot = 0, bool bf16 = false) {
   int rc = check_shape(shape);
   if (rc) return rc;
+  const int elt = bf16 ? 2 : 1;  // bytes per activation / weight element
   if (halo_top < 0 || halo_top > 1 || halo_bot < 0 || halo_bot > 1) return QVAE_ERR_ARG;
   // the input tensor map's largest stride (one batch item) must fit 40 bits
   if (static_cast<double>(shape->T + (carry ? 2 : 0)) * (shape->H + halo_top + halo_bot) * shape->W *
-          shape->Cin >= 1099511627776.0)
+          shape->Cin * elt >= 1099511627776.0)
     return QVAE_ERR_SHAPE;
   const bool acc_mode = acc != nullptr;
   const qvae_shape& s = *shape;
   if (pixels(s) == 0) return QVAE_OK;  // nothing to read or write
-  if (!xq || !wq || (!acc_mode && (!x_scale || !w_scale || !out))) return QVAE_ERR_ARG;
+  if (!xq || !wq || (!acc_mode && !out) || (!acc_mode && !bf16 && (!x_scale || !w_scale))) return QVAE_ERR_ARG;
   if (!aligned16(xq) || !aligned16(wq) || (out && !aligned16(out)) || (acc && !aligned16(acc)))
     return QVAE_ERR_ALIGN;
   int dev;
@@ -307,9 +311,12 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   int sms;
   rc = sm_count(dev, &sms);
   if (rc) return rc;
+  qvae_shape sb = s;  // the geometry in bytes: bf16 is tiled as twice the channels of codes
+  sb.Cin = s.Cin * elt;
   Tiling t;
-  rc = make_tiling(s, &t, sms);
+  rc = make_tiling(sb, &t, sms);
   if (rc) return rc;
+  const int nchunks = (sb.Cin + 127) / 128;  // 128-byte channel chunks
 
   CUtensorMap tmap_x, tmap_w, tmap_out;
   {
@@ -317,19 +324,18 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
     const cuuint64_t h_in = static_cast<cuuint64_t>(s.H) + halo_top + halo_bot;
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W), h_in, t_in,
                                 static_cast<cuuint64_t>(s.N)};
-    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin),
-                                   static_cast<cuuint64_t>(s.W) * s.Cin,
-                                   h_in * s.W * s.Cin,
-                                   t_in * h_in * s.W * s.Cin};
-    const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(qvae::kBoxW),
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin) * elt,
+                                   static_cast<cuuint64_t>(s.W) * s.Cin * elt,
+                                   h_in * s.W * s.Cin * elt,
+                                   t_in * h_in * s.W * s.Cin * elt};
+    const cuuint32_t box[5] = {128u / elt, static_cast<cuuint32_t>(qvae::kBoxW),
                                static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
-    rc = encode_map(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims, strides, box, 5,
-                    CU_TENSOR_MAP_SWIZZLE_128B);
+    rc = encode_map(&tmap_x, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims,
+                    strides, box, 5, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
   }
   {
     // packed weights as rows of 128 bytes: [tap][chunk][Cout] rows
-    const int nchunks = (s.Cin + 127) / 128;
     const cuuint64_t dims[2] = {128u, static_cast<cuuint64_t>(27) * nchunks * s.Cout};
     const cuuint64_t strides[1] = {128u};
     const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(t.pair ? t.NT / 2 : t.NT)};
@@ -367,8 +373,9 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.tiles_h = t.tiles_h;
   a.tiles_n = t.tiles_n;
   a.num_tiles = t.num_tiles;
-  a.nchunks = (s.Cin + 127) / 128;
-  a.last_ksteps = (s.Cin - (a.nchunks - 1) * 128) / 32;
+  a.nchunks = nchunks;
+  a.last_ksteps = (sb.Cin - (nchunks - 1) * 128) / 32;
+  a.chunk_elems = 128 / elt;
   a.SA = t.SA;
   a.SB = t.SB;
   a.acc_stages = t.acc_stages;
@@ -386,13 +393,15 @@ int launch_conv(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
   a.x_scale = x_scale;
   a.w_scale = w_scale;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
-  a.acc_out = acc;
+  a.acc_out = static_cast<int32_t*>(acc);
   a.wait_limit_ns = g_wait_limit_ns;
 
-  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0);
+  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0);
   using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, qvae::ConvArgs);
-  const Kernel kernels[4] = {qvae::conv3d_w8a8_kernel<false, false>, qvae::conv3d_w8a8_kernel<true, false>,
-                             qvae::conv3d_w8a8_kernel<false, true>, qvae::conv3d_w8a8_kernel<true, true>};
+  const Kernel kernels[8] = {qvae::conv3d_w8a8_kernel<false, false>, qvae::conv3d_w8a8_kernel<true, false>,
+                             qvae::conv3d_w8a8_kernel<false, true>,  qvae::conv3d_w8a8_kernel<true, true>,
+                             qvae::conv3d_bf16_kernel<false, false>, qvae::conv3d_bf16_kernel<true, false>,
+                             qvae::conv3d_bf16_kernel<false, true>,  qvae::conv3d_bf16_kernel<true, true>};
   const Kernel kernel = kernels[kidx];
   if (!g_conv_attr_set[dev][kidx]) {
     QVAE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
@@ -664,6 +673,40 @@ int qvae_causal_conv3d_w8a8_carry_acc32(const qvae_shape* shape, const int8_t* x
                      static_cast<cudaStream_t>(stream), true);
 }
 
+size_t qvae_packed_weight_bytes_bf16(int32_t Cin, int32_t Cout) {
+  if (Cin <= 0 || Cout <= 0) return 0;
+  return static_cast<size_t>(27) * ((Cin + 63) / 64) * static_cast<size_t>(Cout) * 128;
+}
+
+int qvae_pack_weights_bf16(int32_t Cin, int32_t Cout, const void* w_bf16, void* w_packed, void* stream) {
+  if (!w_bf16 || !w_packed) return QVAE_ERR_ARG;
+  if (Cin < 32 || Cout < 32 || Cin % 32 || Cout % 32) return QVAE_ERR_SHAPE;
+  if (!aligned16(w_packed)) return QVAE_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nchunks = (Cin + 63) / 64;
+  const int64_t total = static_cast<int64_t>(27) * nchunks * Cout * 64;
+  const int blocks = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 65535));
+  qvae::weight_pack_bf16_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(w_bf16), Cin, Cout, nchunks,
+                                                        static_cast<uint16_t*>(w_packed));
+  QVAE_CUDA(cudaGetLastError());
+  qvae::stream_fence_kernel<<<1, 32, 0, st>>>();  // see the convolution's early weight loads
+  QVAE_CUDA(cudaGetLastError());
+  return QVAE_OK;
+}
+
+int qvae_causal_conv3d_bf16(const qvae_shape* shape, const void* x_bf16, const void* w_packed,
+                            const void* bias_bf16, void* out_bf16, void* stream) {
+  return launch_conv(shape, x_bf16, nullptr, w_packed, nullptr, bias_bf16, out_bf16, nullptr,
+                     static_cast<cudaStream_t>(stream), false, nullptr, 0, 0, true);
+}
+
+int qvae_causal_conv3d_bf16_acc32(const qvae_shape* shape, const void* x_bf16, const void* w_packed,
+                                  float* acc, void* stream) {
+  if (!acc) return QVAE_ERR_ARG;
+  return launch_conv(shape, x_bf16, nullptr, w_packed, nullptr, nullptr, nullptr, acc,
+                     static_cast<cudaStream_t>(stream), false, nullptr, 0, 0, true);
+}
+
 int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
                                   void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -712,12 +755,17 @@ size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {
   return align_up(static_cast<size_t>(max_in), 256) + 256 + kActWorkspace;
 }
 
-// Layer i's output is, element for element, layer i + 1's input (both
-// quantised, same pixels, Cout == next Cin, same pointer).
+// The library runs a layer when it is quantised, or when it is a native-
+// precision layer given bf16 weights packed by qvae_pack_weights_bf16.
+bool runs(const qvae_layer& L) { return L.quantized || L.wq_packed; }
+
+// Layer i's output is, element for element, layer i + 1's input and layer
+// i + 1 is quantised (same pixels, Cout == next Cin, same pointer): layer i's
+// epilogue can take the maximum that layer i + 1's quantiser needs.
 bool feeds_next(const qvae_layer* layers, int32_t n, int32_t i) {
   if (i + 1 >= n) return false;
   const qvae_layer &a = layers[i], &b = layers[i + 1];
-  return a.quantized && b.quantized && a.out == b.x && a.shape.N == b.shape.N && a.shape.T == b.shape.T &&
+  return runs(a) && b.quantized && a.out == b.x && a.shape.N == b.shape.N && a.shape.T == b.shape.T &&
          a.shape.H == b.shape.H && a.shape.W == b.shape.W && a.shape.Cout == b.shape.Cin;
 }
 
@@ -726,10 +774,10 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
   if (n < 0 || (n > 0 && !layers)) return QVAE_ERR_ARG;
   for (int32_t i = 0; i < n; ++i) {
     const qvae_layer& L = layers[i];
-    if (!L.quantized) continue;
+    if (!runs(L)) continue;
     int rc = check_shape(&L.shape);
     if (rc) return rc;
-    if (!L.x || !L.out || !L.wq_packed || !L.w_scale) return QVAE_ERR_ARG;
+    if (!L.x || !L.out || !L.wq_packed || (L.quantized && !L.w_scale)) return QVAE_ERR_ARG;
     if (!aligned16(L.x) || !aligned16(L.out) || !aligned16(L.wq_packed)) return QVAE_ERR_ALIGN;
   }
   const size_t need = qvae_decode_workspace_bytes(layers, n);
@@ -741,8 +789,11 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
     if (rc) return rc;
     if ((rc = sm_count(dev, &sms))) return rc;
     for (int32_t i = 0; i < n; ++i) {
+      if (!runs(layers[i])) continue;
+      qvae_shape sb = layers[i].shape;
+      if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
-      if (layers[i].quantized && (rc = make_tiling(layers[i].shape, &t, sms))) return rc;
+      if ((rc = make_tiling(sb, &t, sms))) return rc;
     }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -757,13 +808,22 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int32_t i = 0; i < n; ++i) {
     const qvae_layer& L = layers[i];
-    if (!L.quantized) continue;
+    if (!runs(L)) continue;
+    const bool feeds = feeds_next(layers, n, i);  // accumulate the next input's absmax
+    uint32_t* next_amax = feeds ? amax_word[(i + 1) & 1] : nullptr;
+    int rc;
+    if (!L.quantized) {
+      // native precision: the bf16 convolution straight from the bf16 input
+      if (next_amax) QVAE_CUDA(cudaMemsetAsync(next_amax, 0, sizeof(uint32_t), st));
+      rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, nullptr, L.bias, L.out, nullptr, st, false, next_amax,
+                       0, 0, true);
+      if (rc) return rc;
+      continue;
+    }
     const int64_t numel = pixels(L.shape) * L.shape.Cin;
     const bool fed = i > 0 && feeds_next(layers, n, i - 1);  // input absmax already accumulated
-    const bool feeds = feeds_next(layers, n, i);            // accumulate the next input's absmax
-    uint32_t* next_amax = feeds ? amax_word[(i + 1) & 1] : nullptr;
-    int rc = fed ? launch_quant_from_amax(L.x, numel, amax_word[i & 1], xq, x_scale, next_amax, st)
-                 : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, next_amax);
+    rc = fed ? launch_quant_from_amax(L.x, numel, amax_word[i & 1], xq, x_scale, next_amax, st)
+             : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, next_amax);
     if (rc) return rc;
     rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
                      next_amax);

@@ -31,6 +31,8 @@ EXPORTS = (
     "qvae_causal_conv3d_w8a8_carry", "qvae_causal_conv3d_w8a8_carry_acc32",
     "qvae_act_absmax", "qvae_act_quant_from_absmax",
     "qvae_causal_conv3d_w8a8_band", "qvae_causal_conv3d_w8a8_band_acc32",
+    "qvae_packed_weight_bytes_bf16", "qvae_pack_weights_bf16", "qvae_causal_conv3d_bf16",
+    "qvae_causal_conv3d_bf16_acc32",
 )
 
 
@@ -81,6 +83,10 @@ def lib():
                                              ctypes.c_int),
             "qvae_causal_conv3d_w8a8_band_acc32": ([ctypes.POINTER(qvae_shape), i32, i32, p, p, p, p],
                                                    ctypes.c_int),
+            "qvae_packed_weight_bytes_bf16": ([i32, i32], sz),
+            "qvae_pack_weights_bf16": ([i32, i32, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_bf16": ([ctypes.POINTER(qvae_shape), p, p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_bf16_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
             "qvae_decode_layers": ([ctypes.POINTER(qvae_layer), i32, p, sz, p], ctypes.c_int),
             "qvae_get_error": ([p], ctypes.c_int),
@@ -291,10 +297,62 @@ def conv_acc32(xq, wq_packed, Cout: int, stream=None):
     return acc
 
 
+# ------------------------------------------------- native-precision layer
+
+def qvae_packed_weight_bytes_bf16(Cin: int, Cout: int) -> int:
+    return int(lib().qvae_packed_weight_bytes_bf16(Cin, Cout))
+
+
+def qvae_pack_weights_bf16(w: torch.Tensor, w_packed: torch.Tensor, stream=None) -> None:
+    Cout, Cin = int(w.shape[0]), int(w.shape[1])
+    _check("qvae_pack_weights_bf16",
+           lib().qvae_pack_weights_bf16(Cin, Cout, _ptr(w), _ptr(w_packed), _stream(stream)))
+
+
+def pack_weights_bf16(w: torch.Tensor, stream=None) -> torch.Tensor:
+    """Allocate and fill the packed bf16 weights of a native-precision layer."""
+    Cout, Cin = int(w.shape[0]), int(w.shape[1])
+    packed = torch.empty(qvae_packed_weight_bytes_bf16(Cin, Cout), dtype=torch.uint8, device=w.device)
+    qvae_pack_weights_bf16(w, packed, stream)
+    return packed
+
+
+def qvae_causal_conv3d_bf16(x: torch.Tensor, w_packed: torch.Tensor, bias: Optional[torch.Tensor],
+                            out: torch.Tensor, stream=None) -> None:
+    shp = shape_of(x, int(out.shape[-1]))
+    _check("qvae_causal_conv3d_bf16",
+           lib().qvae_causal_conv3d_bf16(ctypes.byref(shp), _ptr(x), _ptr(w_packed), _ptr(bias), _ptr(out),
+                                         _stream(stream)))
+
+
+def qvae_causal_conv3d_bf16_acc32(x: torch.Tensor, w_packed: torch.Tensor, acc: torch.Tensor,
+                                  stream=None) -> None:
+    shp = shape_of(x, int(acc.shape[-1]))
+    _check("qvae_causal_conv3d_bf16_acc32",
+           lib().qvae_causal_conv3d_bf16_acc32(ctypes.byref(shp), _ptr(x), _ptr(w_packed), _ptr(acc),
+                                               _stream(stream)))
+
+
+def causal_conv3d_bf16(x, w_packed, bias, Cout: int, stream=None):
+    out = torch.empty(tuple(x.shape[:-1]) + (Cout,), dtype=torch.bfloat16, device=x.device)
+    qvae_causal_conv3d_bf16(x, w_packed, bias, out, stream)
+    return out
+
+
+def conv_bf16_acc32(x, w_packed, Cout: int, stream=None):
+    acc = torch.empty(tuple(x.shape[:-1]) + (Cout,), dtype=torch.float32, device=x.device)
+    qvae_causal_conv3d_bf16_acc32(x, w_packed, acc, stream)
+    return acc
+
+
 # ------------------------------------------------------------ layer chain
 
 def make_layers(specs: Sequence[dict]):
-    """specs: dicts with x, out, wq_packed, w_scale, bias (tensors), quantized (bool)."""
+    """specs: dicts with x, out, wq_packed, w_scale, bias (tensors), quantized (bool).
+
+    A native-precision layer (quantized=False) carries the output of
+    pack_weights_bf16 as wq_packed (the library runs it), or no weights (the
+    library skips it)."""
     arr = (qvae_layer * len(specs))()
     for i, s in enumerate(specs):
         x, out = s["x"], s["out"]
