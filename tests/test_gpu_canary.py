@@ -82,7 +82,8 @@ def test_conv_outputs_stay_inside_their_buffers(q, shape, mode):
             assert_guards(bbuf)
             assert torch.equal(bout.view(torch.int16), ref[:, :, r0:r1].view(torch.int16))
         # a streamed chunk with two carried frames (zero history)
-        xq_ext = torch.cat([torch.zeros_like(xq[:, :2]), xq], 1).contiguous()
+        zeros = torch.zeros((shape.N, 2, shape.H, shape.W, shape.Cin), dtype=torch.int8, device="cuda")
+        xq_ext = torch.cat([zeros, xq], 1).contiguous()
         cout, cbuf = guarded(oshape, torch.bfloat16)
         q.qvae_causal_conv3d_w8a8_carry(xq_ext, s_a, packed, s_w, b, cout)
         assert_guards(cbuf)
