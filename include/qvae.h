@@ -229,6 +229,33 @@ int qvae_causal_conv3d_w8a8_band(const qvae_shape* shape, int32_t halo_top, int3
                                  const int8_t* xq_band, const float* x_scale, const int8_t* wq_packed,
                                  const float* w_scale, const void* bias_bf16, void* out_bf16, void* stream);
 
+/*
+ * The W8A8 convolution quantising its bf16 input itself (the quantise step
+ * fused into the convolution's producer): x is read once, as bf16, by the
+ * convolution, and its codes are made in shared memory -- never written to
+ * device memory.  The codes and the scale are those of qvae_act_absmax_quant
+ * for the maximum *x_amax:
+ *   scale = bf16(*x_amax) / 127,  code = clamp(rint(x / scale), -127, 127),
+ * and the output is that of qvae_causal_conv3d_w8a8 on those codes.
+ *   x_bf16      [N][T][H][W][Cin] bf16.
+ *   x_amax      device uint32: the bf16 magnitude bits of max |x| over the
+ *               tensor (qvae_act_absmax writes it), read after the kernel
+ *               before this call on the stream has finished.
+ *   x_scale_out device fp32, or NULL: receives the activation scale.
+ * A layer is then qvae_act_absmax followed by this call: two passes over x
+ * instead of the absmax, the quantise pass and the codes' write and read.
+ * Same arguments, layout, errors and ordering as qvae_causal_conv3d_w8a8
+ * otherwise (x_bf16, like wq_packed, must not be written by the kernel
+ * launched immediately before this call).
+ */
+int qvae_causal_conv3d_w8a8_fused(const qvae_shape* shape, const void* x_bf16, const uint32_t* x_amax,
+                                  const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
+                                  void* out_bf16, float* x_scale_out, void* stream);
+
+/* The fused convolution writing raw INT32 accumulators [N][T][H][W][Cout]. */
+int qvae_causal_conv3d_w8a8_fused_acc32(const qvae_shape* shape, const void* x_bf16, const uint32_t* x_amax,
+                                        const int8_t* wq_packed, int32_t* acc, void* stream);
+
 /* The row-band convolution writing raw INT32 accumulators [N][T][H][W][Cout]. */
 int qvae_causal_conv3d_w8a8_band_acc32(const qvae_shape* shape, int32_t halo_top, int32_t halo_bot,
                                        const int8_t* xq_band, const int8_t* wq_packed, int32_t* acc,
@@ -297,19 +324,21 @@ typedef struct qvae_layer {
   const void* bias;          /* bf16 [Cout] or NULL */
 } qvae_layer;
 
-/* Workspace bytes qvae_decode_layers needs for these layers. */
+/* Workspace bytes qvae_decode_layers needs (256): the last quantised layer's
+ * activation scale (fp32 at byte 0) and three maximum words. */
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
 
 /*
- * In order on one stream, for each quantised layer: activation absmax +
- * quantise into the workspace, then the W8A8 convolution into `out`; for each
- * native layer with packed bf16 weights: the bf16 convolution into `out`;
- * native layers without weights are skipped.  All layers are validated
- * before anything is launched.  When a layer's `out` is the next layer's `x`
- * and the next layer is quantised (same N, T, H, W and Cout == next Cin), the
- * convolution also accumulates the maximum bf16 magnitude it writes into the
- * workspace and the next layer skips its absmax pass: codes, scales and
- * outputs are the same as layer-by-layer calls.
+ * In order on one stream, for each quantised layer: the activation absmax
+ * into a workspace word, then the fused W8A8 convolution (which quantises x
+ * itself) into `out`; for each native layer with packed bf16 weights: the
+ * bf16 convolution into `out`; native layers without weights are skipped.
+ * All layers are validated before anything is launched.  When a layer's
+ * `out` is the next layer's `x` and the next layer is quantised (same N, T,
+ * H, W and Cout == next Cin), the convolution also accumulates the maximum
+ * bf16 magnitude it writes and the next layer skips its absmax pass: each
+ * quantised layer is then one kernel.  Codes, scales and outputs are the
+ * same as layer-by-layer qvae_act_absmax_quant + qvae_causal_conv3d_w8a8.
  */
 int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
                        size_t workspace_bytes, void* stream);

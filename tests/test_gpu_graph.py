@@ -141,12 +141,14 @@ def _check_chain_against_oracle(q, specs, weights):
     The oracle chain starts from the first input alone: layer k's reference
     input is the oracle's own output of layer k - 1 (the chain is bit-exact,
     so the GPU's input bits must equal it).  For each k the chain is run
-    again on its first k + 1 layers, which leaves layer k's codes and scale
-    in the workspace (codes at offset 0, the scale after the largest input's
-    codes rounded up to 256 bytes); codes, scale, the INT32 accumulators of
-    those codes and the bf16 output are compared element by element.  Layer
-    k's output as the chain writes it when it also feeds layer k + 1 (with
-    the epilogue maximum) is checked as layer k + 1's input."""
+    again on its first k + 1 layers.  The workspace then holds layer k's
+    activation scale (fp32 at byte 0) and its input maximum (word k % 3 at
+    byte 64 + 64 * (k % 3)): for k > 0 the maximum the previous layer's
+    epilogue took over what it wrote.  Maximum, scale, the INT32 accumulators
+    (the fused convolution's accumulator variant on the same input and word)
+    and the bf16 output are compared element by element.  Layer k's output as
+    the chain writes it when it also feeds layer k + 1 (with the epilogue
+    maximum) is checked as layer k + 1's input."""
     import oracle
     ref_in = _np_bits(specs[0]["x"])
     for k, (sp, (packed, s_w, b, Cout)) in enumerate(zip(specs, weights)):
@@ -154,21 +156,20 @@ def _check_chain_against_oracle(q, specs, weights):
         for j in range(k + 1):
             specs[j]["out"].fill_(0)
         layers = q.make_layers(specs[:k + 1])
-        need = q.qvae_decode_workspace_bytes(layers)          # the layout follows these layers
-        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(q.qvae_decode_workspace_bytes(layers), dtype=torch.uint8, device="cuda")
         q.qvae_decode_layers(layers, ws)
         torch.cuda.synchronize()
         assert q.qvae_get_error() == 0
         x_bits = _np_bits(sp["x"])
         assert np.array_equal(x_bits, ref_in), f"layer {k}: input differs from the oracle chain"
         ref = oracle.layer(ref_in, _np_bits(sp["w"]), _np_bits(b))
-        numel = sp["x"].numel()
-        codes = ws[:numel].view(torch.int8).view(sp["x"].shape)
-        xq_bytes = need - 256 - q.qvae_act_workspace_bytes(1)
-        scale = ws[xq_bytes:xq_bytes + 4].view(torch.float32)
-        assert np.array_equal(codes.cpu().numpy(), ref["qx"]), f"layer {k}: codes differ"
+        amax_bits = int(np.array([oracle.act_absmax(ref_in)], np.float32).view(np.uint32)[0] >> 16) & 0x7FFF
+        word = ws[64 + 64 * (k % 3):64 + 64 * (k % 3) + 4].view(torch.int32)
+        assert int(word.item()) == amax_bits, f"layer {k}: input maximum differs"
+        scale = ws[0:4].view(torch.float32)
         assert scale.cpu().numpy().view(np.uint32)[0] == np.array([ref["s_a"]], np.float32).view(np.uint32)[0]
-        acc = q.conv_acc32(codes.contiguous(), packed, Cout)
+        acc = torch.empty(tuple(sp["x"].shape[:-1]) + (Cout,), dtype=torch.int32, device="cuda")
+        q.qvae_causal_conv3d_w8a8_fused_acc32(sp["x"], word.clone(), packed, acc)
         assert np.array_equal(acc.cpu().numpy(), ref["acc"]), f"layer {k}: accumulators differ"
         got = _np_bits(sp["out"])
         assert np.array_equal(got, ref["out"]), f"layer {k}: {np.count_nonzero(got != ref['out'])} outputs differ"

@@ -190,8 +190,8 @@ def test_decode_layers_run_a_native_layer_inside_a_chain(q):
     check_outputs(dev_bits(specs[1]["out"]), r1)
     x2 = dev_bits(specs[2]["x"])
     r2 = oracle.layer(x2, dev_bits(specs[2]["w"]), dev_bits(specs[2]["bias"]))
-    numel = specs[2]["x"].numel()
-    xq_bytes = ws.numel() - 256 - q.qvae_act_workspace_bytes(1)
-    assert np.array_equal(ws[:numel].view(torch.int8).cpu().numpy().reshape(r2["qx"].shape), r2["qx"])
-    assert ws[xq_bytes:xq_bytes + 4].view(torch.float32).item() == r2["s_a"]
+    # layer 2's input maximum, taken by the native layer's epilogue (word 2 % 3), and its scale
+    amax_bits = int(np.array([oracle.act_absmax(x2)], np.float32).view(np.uint32)[0] >> 16) & 0x7FFF
+    assert int(ws[64 + 64 * 2:64 + 64 * 2 + 4].view(torch.int32).item()) == amax_bits
+    assert ws[0:4].view(torch.float32).item() == r2["s_a"]
     assert np.array_equal(dev_bits(specs[2]["out"]), r2["out"])

@@ -389,3 +389,35 @@ def test_conv_right_after_weight_packing(q):
         qw, sw_ref = oracle.quantize_weights(dev_bits(w_dev))
         want = oracle.epilogue(oracle.conv_acc(qx, qw), s_ref, sw_ref, dev_bits(b_dev))
         assert assert_bf16_close(dev_bits(out), want) == 1.0
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_conv_large_accumulators_exact(q, mode):
+    """Accumulators beyond 2^22 in magnitude (codes of +-127 against weights of
+    +-127 over many taps reach 55.7 M for Cin = 384) take the epilogue's other
+    int32 -> float path; a constant image region next to a small-valued one
+    mixes both paths inside one warp.  Every output must still equal the
+    oracle's bit for bit."""
+    shape = synth.LayerShape(384, 192, 20, 24, T=2)
+    g = torch.Generator().manual_seed(99)
+    x = (torch.randn((1, 2, 20, 24, 384), generator=g) * 0.01)
+    x[:, :, :10] = 1.0                                     # codes 127 in the upper half
+    x[:, 1, 5:8, 3:9] = -1.0                               # and a negative patch
+    w = torch.full((192, 384, 3, 3, 3), 0.02)
+    w[::3] *= -1.0                                          # both signs of the maximum
+    w[1::5, ::7] = 0.0013
+    b = (torch.randn(192, generator=g) * 0.01)
+    x, w, b = x.to(torch.bfloat16).cuda(), w.to(torch.bfloat16).cuda(), b.to(torch.bfloat16).cuda()
+    q.qvae_set_conv_tiling(mode=mode)
+    try:
+        packed, s_w = q.quantize_weights(w)
+        xq, s_a = q.act_absmax_quant(x)
+        acc = q.conv_acc32(xq, packed, 192)
+        out = q.causal_conv3d_w8a8(xq, s_a, packed, s_w, b, 192)
+        assert q.qvae_get_error() == 0
+    finally:
+        q.qvae_set_conv_tiling()
+    ref = oracle.layer(dev_bits(x), dev_bits(w), dev_bits(b))
+    assert np.abs(ref["acc"]).max() > 2 ** 22 and np.abs(ref["acc"]).min() < 2 ** 20
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(dev_bits(out), ref["out"])

@@ -71,6 +71,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace qvae {
 
@@ -102,11 +103,23 @@ struct ConvArgs {
   int32_t* acc_out;           // [N,T,H,W,Cout] (accumulator mode)
   uint32_t* out_amax;         // or null: max |bf16 output| (15-bit magnitude) accumulated here
   uint64_t wait_limit_ns;
+  // quantisation in the kernel (fused variant): x is bf16, its codes are made here
+  const uint32_t* x_amax;     // bf16 magnitude bits of max |x| (the scale is bf16(amax) / 127)
+  float* x_scale_out;         // or null: the activation scale is written here
+  int SS;                     // staging slots
+  int stg_rows;               // image rows per staging slot
+  int stg_groups;             // staging slots per activation box: (16 * MS + 2) / stg_rows
+  uint32_t stg_slot_bytes;    // stg_rows x 10 pixels x 128 channels x 2 bytes
+  uint32_t* zero_word;        // or null: a word set to zero (for a later layer's maximum)
 };
 
 constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
 constexpr int kConvThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
+constexpr int kCvtWarps = 2;                        // quantising warps of the fused variant
+constexpr int kConvThreadsFused = kConvThreads + 32 * kCvtWarps;
 constexpr int kMaxStages = 12;
+constexpr int kMaxStgSlots = 8;
+constexpr uint32_t kStgPixelBytes = 256;            // 128 bf16 channels of one pixel
 constexpr uint32_t kEpiBufBytes = 2048;    // one epilogue staging buffer: 32 pixels x 64 B
 constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
 
@@ -156,7 +169,7 @@ struct MmaRings {
 // starts) while the later sub-tiles still run, and sub-tile s of the next
 // tile starts as soon as its epilogue has released it.  Returns false when a
 // wait gave up (abort or time limit).
-template <bool kBf16, bool kPair, int kMS, int kG>
+template <bool kBf16, bool kPair, bool kFuse, int kMS, int kG>
 __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
                                                volatile int* abort_flag, uint64_t limit, int first_tile,
                                                int tile_step, uint32_t rank, bool& issued) {
@@ -217,7 +230,12 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
     uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
     for (int kb = 0; kb < nkb; ++kb) {
       const int ch = kb % a.nchunks;
-      if (!mbar_wait(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) return false;
+      // the fused variant's A stages are written by threads of both CTAs of a pair
+      if (kFuse && kPair) {
+        if (!mbar_wait_cluster(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) return false;
+      } else if (!mbar_wait(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) {
+        return false;
+      }
       tc_fence_after();
       const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
       const uint64_t a_stage = a_desc0 + as * a_stage16;
@@ -316,7 +334,14 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
 // shared memory both are 128-byte lines per pixel -- 128 codes or 64 bf16
 // channels -- and one MMA step consumes 32 bytes of K, so the tiling, the
 // rings and the tap offsets are the same.
-template <bool kBf16, bool kAcc32, bool kPair>
+//
+// kFuse (INT8 only): x arrives as bf16 and is quantised inside the kernel.
+// Two more warps stream row groups of the bf16 input box into a small staging
+// ring by TMA and write the codes of each 16-channel group, in the MMA's
+// swizzled layout, into the activation ring -- the same codes as the
+// activation quantiser, with the scale bf16(amax) / 127 taken from one device
+// word.  The producer then loads weights only.
+template <bool kBf16, bool kAcc32, bool kPair, bool kFuse>
 __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w,
                                             const CUtensorMap& tmap_out, const ConvArgs& a) {
   extern __shared__ uint8_t smem_raw[];
@@ -326,12 +351,14 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
 
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
-  const uint32_t epi_stage = b_ring + a.SB * a.b_stage_bytes;  // 1024-aligned
+  const uint32_t stg_ring = b_ring + a.SB * a.b_stage_bytes;                     // fused: bf16 row groups
+  const uint32_t epi_stage = stg_ring + (kFuse ? a.SS * a.stg_slot_bytes : 0u);  // 1024-aligned
   const uint32_t bars = epi_stage + kEpiWarps * a.epi_bufs * kEpiBufBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 8 * kAccBars;
-  const uint32_t drain_bar = acc_empty + 8 * kAccBars;
+  const uint32_t stg_full = acc_empty + 8 * kAccBars, stg_empty = stg_full + 8 * kMaxStgSlots;
+  const uint32_t drain_bar = stg_empty + 8 * kMaxStgSlots;
   uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
   volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -352,8 +379,15 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
   if (threadIdx.x == 64 && !kAcc32) prefetch_tmap(&tmap_out);
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.SA; ++i) {
-      mbar_init(a_full + 8 * i, 1);
+      // fused: one arrive per quantising warp (of both CTAs of a pair)
+      mbar_init(a_full + 8 * i, kFuse ? kCvtWarps * (kPair ? 2 : 1) : 1);
       mbar_init(a_empty + 8 * i, 1);
+    }
+    if (kFuse) {
+      for (int i = 0; i < a.SS; ++i) {
+        mbar_init(stg_full + 8 * i, 1);
+        mbar_init(stg_empty + 8 * i, kCvtWarps);
+      }
     }
     for (int i = 0; i < a.SB; ++i) {
       mbar_init(b_full + 8 * i, 1);
@@ -423,11 +457,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         if (!waited) {
           for (; preissued < a.SB && preissued < ngrp; ++preissued)
             if (!load_b(c, kt, ch, preissued)) goto producer_done;
-          grid_dependency_wait();
+          if (!kFuse) grid_dependency_wait();
           waited = true;
         }
-        if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
-        {
+        if (!kFuse) {
+          if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
           const uint32_t bar = a_full + 8 * as;
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
           if (kPair) {
@@ -437,10 +471,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
             tma_load_5d(a_ring + as * a.a_stage_bytes, &tmap_x, bar, ch * a.chunk_elems, c.w0 - 1,
                         c.h0 - 1 + a.halo_top, frame, c.n);
           }
+          a_armed |= 1u << as;
+          a_par = (a_par & ~(1u << as)) | (ap << as);
+          if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
         }
-        a_armed |= 1u << as;
-        a_par = (a_par & ~(1u << as)) | (ap << as);
-        if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
+        (void)frame;
         for (int i = preissued; i < ngrp; ++i)
           if (!load_b(c, kt, ch, i)) goto producer_done;
         preissued = 0;
@@ -463,9 +498,8 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     bool issued = false;
     bool ok;
     auto run = [&](auto ms, auto g) {
-      return mma_issue_loop<kBf16, kPair, decltype(ms)::value, decltype(g)::value>(a, r, abort_flag, limit,
-                                                                                  first_tile, tile_step, rank,
-                                                                                  issued);
+      return mma_issue_loop<kBf16, kPair, kFuse, decltype(ms)::value, decltype(g)::value>(
+          a, r, abort_flag, limit, first_tile, tile_step, rank, issued);
     };
     using G1 = std::integral_constant<int, 1>;
     using G3 = std::integral_constant<int, 3>;
@@ -499,6 +533,141 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       }
       mbar_wait(drain_bar, 0, &dummy, limit, kErrTimeoutDrain);
     }
+  } else if (kFuse && warp >= 2 + kEpiWarps) {
+    // ----------------------------------------------------------- quantisers
+    // The activation boxes of the fused variant, in the MMA's order: each
+    // box (tile, temporal tap, 128-channel chunk) is 16*MS + 2 rows x 10
+    // columns of bf16 pixels, brought in as row groups of stg_rows rows by
+    // TMA into the staging ring (lane 0 of the first quantising warp keeps
+    // SS groups in flight) and turned into codes, 16 channels per item, in
+    // the 128-byte-swizzled K-major layout of the activation ring.  Rows and
+    // columns beyond the image arrive as zeros from the tensor map and give
+    // code 0.  When a box is complete, each warp fences its shared-memory
+    // writes for the tensor cores and arrives on the (leader's) a_full.
+    const int cw = warp - (2 + kEpiWarps);
+    const int ct = cw * 32 + lane;
+    const bool pf_thread = cw == 0 && lane == 0;
+    struct Pos {
+      int tile, kb, g, nkb, kt_lo;
+      TileCoord c;
+    };
+    auto start = [&](Pos& p, int tile) {
+      p.tile = tile;
+      p.kb = 0;
+      p.g = 0;
+      if (tile < a.num_tiles) {
+        p.c = decode_tile<kPair>(a, tile, rank);
+        p.kt_lo = (a.carry || p.c.t >= 2) ? 0 : 2 - p.c.t;
+        p.nkb = (3 - p.kt_lo) * a.nchunks;
+      }
+    };
+    auto advance = [&](Pos& p) {
+      if (++p.g < a.stg_groups) return;
+      p.g = 0;
+      if (++p.kb < p.nkb) return;
+      start(p, p.tile + tile_step);
+    };
+    uint32_t stg_armed = 0, stg_par = 0;
+    // issue the TMA load of position p into staging slot `slot` (use parity `par`)
+    auto issue = [&](const Pos& p, uint32_t slot) {
+      const int kt = p.kt_lo + p.kb / a.nchunks, ch = p.kb % a.nchunks;
+      const int frame = p.c.t + kt - 2 + 2 * a.carry;
+      const uint32_t bar = stg_full + 8 * slot;
+      mbar_arrive_expect_tx(bar, a.stg_slot_bytes);
+      tma_load_5d(stg_ring + slot * a.stg_slot_bytes, &tmap_x, bar, ch * 128, p.c.w0 - 1,
+                  p.c.h0 - 1 + a.halo_top + p.g * a.stg_rows, frame, p.c.n);
+    };
+    grid_dependency_wait();  // x and its maximum are final
+    const float sa = __fdiv_rn(bf16_bits_to_f32(__ldcg(a.x_amax) & 0x7FFFu) * 1.0f, 127.0f);  // clip ratio 1.0
+    const Quantizer z = make_quantizer(sa);
+    const bool zero_scale = sa == 0.0f;
+    if (ct == 0 && blockIdx.x == 0) {
+      if (a.x_scale_out) *a.x_scale_out = sa;
+      if (a.zero_word) *a.zero_word = 0u;
+    }
+    Pos cur, pf;
+    start(cur, first_tile);
+    start(pf, first_tile);
+    if (pf_thread) {
+      for (uint32_t k = 0; k < static_cast<uint32_t>(a.SS) && pf.tile < a.num_tiles; ++k) {
+        issue(pf, k);
+        stg_armed |= 1u << k;
+        advance(pf);
+      }
+    }
+    uint32_t slot = 0, sp = 0, as = 0, ap = 0;
+    const int lines = a.stg_rows * kBoxW;
+    bool ok = true;
+    while (ok && cur.tile < a.num_tiles) {
+      const int ch = cur.kb % a.nchunks;
+      const int nu = (ch == a.nchunks - 1) ? 2 * a.last_ksteps : 8;  // 16-channel groups the MMA reads
+      const uint32_t a_st = a_ring + as * a.a_stage_bytes;
+      // every lane waits (so that each observes the copies it reads); the
+      // warp leaves together if any lane's wait gave up
+      bool waited = cur.g != 0 || mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutConvert);
+      waited = waited && mbar_wait(stg_full + 8 * slot, sp, abort_flag, limit, kErrTimeoutConvert);
+      if (!__all_sync(0xFFFFFFFFu, waited)) {
+        ok = false;
+        break;
+      }
+      const uint32_t src = stg_ring + slot * a.stg_slot_bytes;
+      const int line0 = cur.g * lines;
+      for (int it = ct; it < lines * nu; it += 32 * kCvtWarps) {
+        const int i = it / nu, u = it - i * nu;
+        const int L = line0 + i;
+        uint4 lo, hi;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w)
+                     : "r"(src + i * kStgPixelBytes + u * 32u));
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                     : "r"(src + i * kStgPixelBytes + u * 32u + 16u));
+        const uint4 q = quant16(z, zero_scale, lo, hi);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         a_st + static_cast<uint32_t>(L) * 128u + ((static_cast<uint32_t>(u) ^ (L & 7u)) << 4)),
+                     "r"(q.x), "r"(q.y), "r"(q.z), "r"(q.w)
+                     : "memory");
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(stg_empty + 8 * slot);
+      if (pf_thread) {
+        // refill this slot with the group SS positions ahead, once both warps are done with it
+        if (pf.tile < a.num_tiles) {
+          if (!mbar_wait(stg_empty + 8 * slot, sp, abort_flag, limit, kErrTimeoutConvert)) {
+            stg_armed &= ~(1u << slot);
+            ok = false;
+          } else {
+            issue(pf, slot);
+            stg_par = (stg_par & ~(1u << slot)) | ((sp ^ 1u) << slot);
+            advance(pf);
+          }
+        } else {
+          stg_armed &= ~(1u << slot);
+        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (++slot == static_cast<uint32_t>(a.SS)) { slot = 0; sp ^= 1; }
+      if (cur.g == a.stg_groups - 1) {
+        // the box is complete: make the codes visible to the tensor cores
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair) {
+            mbar_arrive_cluster(map_to_cta(a_full + 8 * as, 0));
+          } else {
+            mbar_arrive(a_full + 8 * as);
+          }
+        }
+        if (++as == static_cast<uint32_t>(a.SA)) { as = 0; ap ^= 1; }
+      }
+      advance(cur);
+    }
+    if (pf_thread && *abort_flag) {
+      // let the staging loads still in flight land before the CTA exits
+      int dummy = 0;
+      for (int i = 0; i < a.SS; ++i)
+        if (stg_armed >> i & 1) mbar_wait(stg_full + 8 * i, stg_par >> i & 1, &dummy, limit, kErrTimeoutDrain);
+    }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // A warp may read only the TMEM lane quarter warp % 4; lane quarter q holds
@@ -528,7 +697,9 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     // lets the previous tile's slices finish reading the old table.
     auto fill_table = [&](int co0) {
       named_barrier_sync(1, 32 * kEpiWarps);
-      const float sa = kBf16 ? 1.0f : *a.x_scale;
+      const float sa = kBf16   ? 1.0f
+                       : kFuse ? __fdiv_rn(bf16_bits_to_f32(__ldcg(a.x_amax) & 0x7FFFu) * 1.0f, 127.0f)
+                               : *a.x_scale;
       for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
         sc[j] = kBf16 ? 1.0f : __fmul_rn(sa, a.w_scale[co0 + j]);
         bi[j] = a.bias ? __bfloat162float(a.bias[co0 + j]) : 0.0f;
@@ -691,7 +862,15 @@ template <bool kAcc32, bool kPair>
 __global__ void __launch_bounds__(kConvThreads, 1)
     conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
-  conv3d_body<false, kAcc32, kPair>(tmap_x, tmap_w, tmap_out, a);
+  conv3d_body<false, kAcc32, kPair, false>(tmap_x, tmap_w, tmap_out, a);
+}
+
+// W8A8 convolution quantising its bf16 input in the kernel (scale from a maximum word).
+template <bool kAcc32, bool kPair>
+__global__ void __launch_bounds__(kConvThreadsFused, 1)
+    conv3d_w8a8_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                             const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
+  conv3d_body<false, kAcc32, kPair, true>(tmap_x, tmap_w, tmap_out, a);
 }
 
 // Native-precision convolution: bf16 values, fp32 accumulators, + bias.
@@ -699,7 +878,7 @@ template <bool kAcc32, bool kPair>
 __global__ void __launch_bounds__(kConvThreads, 1)
     conv3d_bf16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
-  conv3d_body<true, kAcc32, kPair>(tmap_x, tmap_w, tmap_out, a);
+  conv3d_body<true, kAcc32, kPair, false>(tmap_x, tmap_w, tmap_out, a);
 }
 
 // A wait that nothing satisfies: checks that a bounded wait gives up, raises

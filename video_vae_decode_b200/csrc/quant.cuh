@@ -137,10 +137,46 @@ __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __
   }
 }
 
+// Four codes from four bf16 values, two at a time on the packed fp32 pipe
+// (mul / fma .rn.f32x2): the same correctly rounded quotient as code_byte
+// (q0 = RN(v r), e = fma(-q0, s, v), q = fma(e, r, q0)) and the same
+// round-half-even add of 1.5 * 2^23.  No clamp: |v| <= amax and
+// s = RN(amax / 127) >= (amax / 127)(1 - 2^-24) give |v / s| < 127.00001, whose
+// rounded quotient rounds to at most 127.  For normal, non-zero scales only
+// (make_quantizer's reciprocal path).
+__device__ __forceinline__ uint32_t quant4_x2(const Quantizer& z, uint32_t w0, uint32_t w1) {
+  const uint64_t rr = (static_cast<uint64_t>(__float_as_uint(z.r)) << 32) | __float_as_uint(z.r);
+  const uint64_t ns = (static_cast<uint64_t>(__float_as_uint(-z.s)) << 32) | __float_as_uint(-z.s);
+  const uint64_t mg = 0x4B4000004B400000ull;  // 1.5 * 2^23 in both halves
+  // (v0, v1) in the low / high halves: the bf16 values widened to fp32
+  const uint64_t va = (static_cast<uint64_t>(w0 & 0xFFFF0000u) << 32) | (w0 << 16);
+  const uint64_t vb = (static_cast<uint64_t>(w1 & 0xFFFF0000u) << 32) | (w1 << 16);
+  uint64_t qa, qb, ea, eb;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(qa) : "l"(va), "l"(rr));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(qb) : "l"(vb), "l"(rr));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ea) : "l"(qa), "l"(ns), "l"(va));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(eb) : "l"(qb), "l"(ns), "l"(vb));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(qa) : "l"(ea), "l"(rr), "l"(qa));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(qb) : "l"(eb), "l"(rr), "l"(qb));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(qa) : "l"(qa), "l"(mg));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(qb) : "l"(qb), "l"(mg));
+  // low bytes of the four sums, in order v0, v1 (from w0), v2, v3 (from w1)
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(qa), static_cast<uint32_t>(qa >> 32), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(qb), static_cast<uint32_t>(qb >> 32), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
 // 16 bf16 values (two 16-byte vectors) -> 16 codes (one 16-byte vector).
 __device__ __forceinline__ uint4 quant16(const Quantizer& z, bool zero, const uint4& a, const uint4& b) {
   if (zero) return make_uint4(0u, 0u, 0u, 0u);
   return make_uint4(quant4(z, a.x, a.y), quant4(z, a.z, a.w), quant4(z, b.x, b.y), quant4(z, b.z, b.w));
+}
+
+// quant16 on the packed fp32 pipe (normal scales; tiny scales take quant16).
+__device__ __forceinline__ uint4 quant16_x2(const Quantizer& z, bool zero, const uint4& a, const uint4& b) {
+  if (zero) return make_uint4(0u, 0u, 0u, 0u);
+  if (z.exact) return quant16(z, false, a, b);
+  return make_uint4(quant4_x2(z, a.x, a.y), quant4_x2(z, a.z, a.w), quant4_x2(z, b.x, b.y), quant4_x2(z, b.z, b.w));
 }
 
 // Pass 2: reduce the partial maxima (or read the one maximum the previous

@@ -34,8 +34,8 @@ std::atomic<int32_t> g_cta_limit{0};    // cap on the conv grid (0 = one CTA per
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
-bool g_conv_attr_set[kMaxDevices][8] = {};
-int g_max_clusters[kMaxDevices] = {0};
+bool g_conv_attr_set[kMaxDevices][12] = {};
+int g_max_clusters[kMaxDevices][2] = {};  // per device, per thread count (plain, fused)
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
 
@@ -88,6 +88,8 @@ struct Tiling {
   int MS, NT, SA, SB, acc_stages, G;
   bool split;    // per-sub-tile accumulator hand-off
   int epi_bufs;  // epilogue staging buffers per warp
+  bool fuse;     // quantisation in the kernel: a bf16 staging ring of SS row groups
+  int SS;
   uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
   int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
   double est_cycles;
@@ -95,9 +97,13 @@ struct Tiling {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+constexpr int kStgRows = 2;  // image rows per staging slot of the fused variant (divides 16 * MS + 2)
+constexpr uint32_t kStgSlotBytes = kStgRows * qvae::kBoxW * qvae::kStgPixelBytes;
+
 uint32_t smem_needed(const Tiling& t) {
-  const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 8;
-  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + qvae::kEpiWarps * t.epi_bufs * qvae::kEpiBufBytes +
+  const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 2 * 8 * qvae::kMaxStgSlots + 8;
+  return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + (t.fuse ? t.SS * kStgSlotBytes : 0u) +
+         qvae::kEpiWarps * t.epi_bufs * qvae::kEpiBufBytes +
          bars +
          16 + 16 + 2 * t.NT * 4;
 }
@@ -107,7 +113,19 @@ uint32_t smem_needed(const Tiling& t) {
 // buffers per warp, else the best that fits.  `want_sb`: a weight ring depth
 // to reach first with one staging buffer if it does not fit with two (the
 // sub-tile hand-off needs a whole chunk's stages).
+bool fit_stages_ss(Tiling* t, int want_sb);
+
 bool fit_stages(Tiling* t, int want_sb = 0) {
+  if (!t->fuse) {
+    t->SS = 0;
+    return fit_stages_ss(t, want_sb);
+  }
+  for (t->SS = 4; t->SS >= 2; t->SS -= 2)
+    if (fit_stages_ss(t, want_sb)) return true;
+  return false;
+}
+
+bool fit_stages_ss(Tiling* t, int want_sb) {
   if (g_force[2] || g_force[3]) {
     t->SA = g_force[2] ? g_force[2].load() : 2;
     t->SB = g_force[3] ? g_force[3].load() : 4;
@@ -157,8 +175,9 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   return (waves * per_tile + tail) * (t.pair ? 0.98 : 1.0);
 }
 
-int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t) {
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse) {
   if (G != 1 && !(G == 3 && MS <= 2)) return QVAE_ERR_ARG;  // kernel instantiations
+  t->fuse = fuse;
   t->pair = pair;
   t->MS = MS;
   t->NT = NT;
@@ -193,7 +212,7 @@ int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms
   return QVAE_OK;
 }
 
-int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148) {
+int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false) {
   bool found = false;
   for (int mode = 1; mode <= 2; ++mode) {
     if (g_force[4] && mode != g_force[4]) continue;
@@ -205,7 +224,7 @@ int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148) {
         for (int g = 1; g <= 3; g += 2) {
           if (g_force[5] && g != g_force[5]) continue;
           Tiling u;
-          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u) != QVAE_OK) continue;
+          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u, fuse) != QVAE_OK) continue;
           u.est_cycles = estimate_cycles(s, u, sms);
           if (!found || u.est_cycles < t->est_cycles) {
             *t = u;
@@ -287,22 +306,30 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
 // bf16: the native-precision convolution -- xq holds bf16 values, wq the bf16
 // packing, acc (accumulator mode) receives fp32 sums; no scales.  It is tiled
 // as the INT8 convolution of twice the channels (the same bytes per pixel).
+// x_amax != null: the fused W8A8 variant -- xq holds the bf16 input, quantised
+// in the kernel with the scale bf16(*x_amax) / 127; x_scale_out (nullable)
+// receives that scale; zero_word (nullable) is set to zero by the kernel.
 int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
                 const void* wq, const float* w_scale, const void* bias, void* out, void* acc,
                 cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr, int halo_top = 0,
-                int halo_bot = 0, bool bf16 = false) {
+                int halo_bot = 0, bool bf16 = false, const uint32_t* x_amax = nullptr,
+                float* x_scale_out = nullptr, uint32_t* zero_word = nullptr) {
   int rc = check_shape(shape);
   if (rc) return rc;
-  const int elt = bf16 ? 2 : 1;  // bytes per activation / weight element
+  const bool fuse = x_amax != nullptr;
+  if (fuse && bf16) return QVAE_ERR_ARG;
+  const int elt = bf16 ? 2 : 1;            // bytes per operand element in shared memory
+  const int x_elt = (bf16 || fuse) ? 2 : 1;  // bytes per input element in global memory
   if (halo_top < 0 || halo_top > 1 || halo_bot < 0 || halo_bot > 1) return QVAE_ERR_ARG;
   // the input tensor map's largest stride (one batch item) must fit 40 bits
   if (static_cast<double>(shape->T + (carry ? 2 : 0)) * (shape->H + halo_top + halo_bot) * shape->W *
-          shape->Cin * elt >= 1099511627776.0)
+          shape->Cin * x_elt >= 1099511627776.0)
     return QVAE_ERR_SHAPE;
   const bool acc_mode = acc != nullptr;
   const qvae_shape& s = *shape;
   if (pixels(s) == 0) return QVAE_OK;  // nothing to read or write
-  if (!xq || !wq || (!acc_mode && !out) || (!acc_mode && !bf16 && (!x_scale || !w_scale))) return QVAE_ERR_ARG;
+  if (!xq || !wq || (!acc_mode && !out) || (!acc_mode && !bf16 && ((!x_scale && !fuse) || !w_scale)))
+    return QVAE_ERR_ARG;
   if (!aligned16(xq) || !aligned16(wq) || (out && !aligned16(out)) || (acc && !aligned16(acc)))
     return QVAE_ERR_ALIGN;
   int dev;
@@ -314,7 +341,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   qvae_shape sb = s;  // the geometry in bytes: bf16 is tiled as twice the channels of codes
   sb.Cin = s.Cin * elt;
   Tiling t;
-  rc = make_tiling(sb, &t, sms);
+  rc = make_tiling(sb, &t, sms, fuse);
   if (rc) return rc;
   const int nchunks = (sb.Cin + 127) / 128;  // 128-byte channel chunks
 
@@ -324,14 +351,21 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
     const cuuint64_t h_in = static_cast<cuuint64_t>(s.H) + halo_top + halo_bot;
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.Cin), static_cast<cuuint64_t>(s.W), h_in, t_in,
                                 static_cast<cuuint64_t>(s.N)};
-    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin) * elt,
-                                   static_cast<cuuint64_t>(s.W) * s.Cin * elt,
-                                   h_in * s.W * s.Cin * elt,
-                                   t_in * h_in * s.W * s.Cin * elt};
-    const cuuint32_t box[5] = {128u / elt, static_cast<cuuint32_t>(qvae::kBoxW),
-                               static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
-    rc = encode_map(&tmap_x, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims,
-                    strides, box, 5, CU_TENSOR_MAP_SWIZZLE_128B);
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.Cin) * x_elt,
+                                   static_cast<cuuint64_t>(s.W) * s.Cin * x_elt,
+                                   h_in * s.W * s.Cin * x_elt,
+                                   t_in * h_in * s.W * s.Cin * x_elt};
+    if (fuse) {
+      // bf16 row groups of the box for the staging ring: 128 channels x 10 columns x kStgRows rows
+      const cuuint32_t box[5] = {128u, static_cast<cuuint32_t>(qvae::kBoxW), static_cast<cuuint32_t>(kStgRows), 1u, 1u};
+      rc = encode_map(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xq, dims, strides, box, 5,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+      const cuuint32_t box[5] = {128u / elt, static_cast<cuuint32_t>(qvae::kBoxW),
+                                 static_cast<cuuint32_t>(t.MS * qvae::kTileRows + 2), 1u, 1u};
+      rc = encode_map(&tmap_x, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, dims,
+                      strides, box, 5, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (rc) return rc;
   }
   {
@@ -395,13 +429,24 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.acc_out = static_cast<int32_t*>(acc);
   a.wait_limit_ns = g_wait_limit_ns;
+  a.x_amax = x_amax;
+  a.x_scale_out = x_scale_out;
+  a.zero_word = zero_word;
+  a.SS = t.SS;
+  a.stg_rows = kStgRows;
+  a.stg_groups = (t.MS * qvae::kTileRows + 2) / kStgRows;
+  a.stg_slot_bytes = kStgSlotBytes;
 
-  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0);
+  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0) + (fuse ? 8 : 0);
   using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, qvae::ConvArgs);
-  const Kernel kernels[8] = {qvae::conv3d_w8a8_kernel<false, false>, qvae::conv3d_w8a8_kernel<true, false>,
-                             qvae::conv3d_w8a8_kernel<false, true>,  qvae::conv3d_w8a8_kernel<true, true>,
-                             qvae::conv3d_bf16_kernel<false, false>, qvae::conv3d_bf16_kernel<true, false>,
-                             qvae::conv3d_bf16_kernel<false, true>,  qvae::conv3d_bf16_kernel<true, true>};
+  const Kernel kernels[12] = {
+      qvae::conv3d_w8a8_kernel<false, false>,       qvae::conv3d_w8a8_kernel<true, false>,
+      qvae::conv3d_w8a8_kernel<false, true>,        qvae::conv3d_w8a8_kernel<true, true>,
+      qvae::conv3d_bf16_kernel<false, false>,       qvae::conv3d_bf16_kernel<true, false>,
+      qvae::conv3d_bf16_kernel<false, true>,        qvae::conv3d_bf16_kernel<true, true>,
+      qvae::conv3d_w8a8_fused_kernel<false, false>, qvae::conv3d_w8a8_fused_kernel<true, false>,
+      qvae::conv3d_w8a8_fused_kernel<false, true>,  qvae::conv3d_w8a8_fused_kernel<true, true>};
+  const int threads = fuse ? qvae::kConvThreadsFused : qvae::kConvThreads;
   const Kernel kernel = kernels[kidx];
   if (!g_conv_attr_set[dev][kidx]) {
     QVAE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
@@ -409,10 +454,11 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   }
   int grid;
   if (t.pair) {
-    if (g_max_clusters[dev] == 0) {
+    int& max_clusters = g_max_clusters[dev][fuse ? 1 : 0];
+    if (max_clusters == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * sms);
-      cfg.blockDim = dim3(qvae::kConvThreads);
+      cfg.blockDim = dim3(threads);
       cfg.dynamicSmemBytes = kSmemLimit;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -423,10 +469,10 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
       cfg.numAttrs = 1;
       int n = 0;
       QVAE_CUDA(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg));
-      g_max_clusters[dev] = std::max(n, 1);
+      max_clusters = std::max(n, 1);
     }
     const int cta_limit = g_cta_limit.load();
-    int clusters = std::min(t.num_tiles, g_max_clusters[dev]);
+    int clusters = std::min(t.num_tiles, max_clusters);
     if (cta_limit > 0) clusters = std::max(1, std::min(clusters, cta_limit / 2));
     grid = 2 * clusters;
   } else {
@@ -434,7 +480,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
     grid = std::min(t.num_tiles, sms);
     if (cta_limit > 0) grid = std::min(grid, cta_limit);
   }
-  QVAE_CUDA(launch_dependent(kernel, grid, qvae::kConvThreads, t.smem_bytes, stream, t.pair ? 2 : 1, tmap_x,
+  QVAE_CUDA(launch_dependent(kernel, grid, threads, t.smem_bytes, stream, t.pair ? 2 : 1, tmap_x,
                              tmap_w, tmap_out, a));
   return QVAE_OK;
 }
@@ -515,8 +561,6 @@ int launch_quant_from_amax(const void* x, int64_t numel, const uint32_t* amax, i
   QVAE_CUDA(cudaGetLastError());
   return QVAE_OK;
 }
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
@@ -707,6 +751,21 @@ int qvae_causal_conv3d_bf16_acc32(const qvae_shape* shape, const void* x_bf16, c
                      static_cast<cudaStream_t>(stream), false, nullptr, 0, 0, true);
 }
 
+int qvae_causal_conv3d_w8a8_fused(const qvae_shape* shape, const void* x_bf16, const uint32_t* x_amax,
+                                  const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
+                                  void* out_bf16, float* x_scale_out, void* stream) {
+  if (!x_amax) return QVAE_ERR_ARG;
+  return launch_conv(shape, x_bf16, nullptr, wq_packed, w_scale, bias_bf16, out_bf16, nullptr,
+                     static_cast<cudaStream_t>(stream), false, nullptr, 0, 0, false, x_amax, x_scale_out);
+}
+
+int qvae_causal_conv3d_w8a8_fused_acc32(const qvae_shape* shape, const void* x_bf16, const uint32_t* x_amax,
+                                        const int8_t* wq_packed, int32_t* acc, void* stream) {
+  if (!x_amax || !acc) return QVAE_ERR_ARG;
+  return launch_conv(shape, x_bf16, nullptr, wq_packed, nullptr, nullptr, nullptr, acc,
+                     static_cast<cudaStream_t>(stream), false, nullptr, 0, 0, false, x_amax);
+}
+
 int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq, float* x_scale,
                                   void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -746,13 +805,13 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
   return QVAE_OK;
 }
 
+// Workspace of qvae_decode_layers: the activation scale of the last quantised
+// layer (fp32 at byte 0) and three 32-bit maximum words (bytes 64, 128, 192).
+constexpr size_t kDecodeWorkspace = 256;
+
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {
   if (!layers || n < 0) return 0;
-  int64_t max_in = 0;
-  for (int32_t i = 0; i < n; ++i)
-    if (layers[i].quantized)
-      max_in = std::max<int64_t>(max_in, pixels(layers[i].shape) * layers[i].shape.Cin);
-  return align_up(static_cast<size_t>(max_in), 256) + 256 + kActWorkspace;
+  return kDecodeWorkspace;
 }
 
 // The library runs a layer when it is quantised, or when it is a native-
@@ -793,40 +852,48 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       qvae_shape sb = layers[i].shape;
       if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
-      if ((rc = make_tiling(sb, &t, sms))) return rc;
+      if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0))) return rc;
     }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t xq_bytes = need - 256 - kActWorkspace;
-  int8_t* xq = reinterpret_cast<int8_t*>(ws);
-  float* x_scale = reinterpret_cast<float*>(ws + xq_bytes);
-  // two words of the 256-byte gap: the absmax of layer i's input, accumulated
-  // by layer i - 1's convolution when it writes that input (alternating)
-  uint32_t* amax_word[2] = {reinterpret_cast<uint32_t*>(ws + xq_bytes + 64),
-                            reinterpret_cast<uint32_t*>(ws + xq_bytes + 128)};
-  void* partial = ws + xq_bytes + 256;
+  float* x_scale = reinterpret_cast<float*>(ws);
+  // Layer i reads its input maximum from word i % 3, accumulates its output's
+  // maximum (when that output feeds the next quantised layer) into word
+  // (i + 1) % 3, and a fused convolution clears word (i + 2) % 3: the word
+  // layer i + 1 will accumulate into, which nothing reads or writes from the
+  // moment layer i starts (layer i - 1, its last reader, has finished).
+  uint32_t* word[3] = {reinterpret_cast<uint32_t*>(ws + 64), reinterpret_cast<uint32_t*>(ws + 128),
+                       reinterpret_cast<uint32_t*>(ws + 192)};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n > 0) QVAE_CUDA(cudaMemsetAsync(ws + 64, 0, 192, st));
+  bool next_cleared = true;  // the word this layer accumulates into is zero
   for (int32_t i = 0; i < n; ++i) {
     const qvae_layer& L = layers[i];
-    if (!runs(L)) continue;
-    const bool feeds = feeds_next(layers, n, i);  // accumulate the next input's absmax
-    uint32_t* next_amax = feeds ? amax_word[(i + 1) & 1] : nullptr;
+    if (!runs(L)) {
+      next_cleared = false;
+      continue;
+    }
+    const bool feeds = feeds_next(layers, n, i);
+    uint32_t* in_word = word[i % 3];
+    uint32_t* out_word = feeds ? word[(i + 1) % 3] : nullptr;
+    if (out_word && !next_cleared) QVAE_CUDA(cudaMemsetAsync(out_word, 0, sizeof(uint32_t), st));
     int rc;
     if (!L.quantized) {
       // native precision: the bf16 convolution straight from the bf16 input
-      if (next_amax) QVAE_CUDA(cudaMemsetAsync(next_amax, 0, sizeof(uint32_t), st));
-      rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, nullptr, L.bias, L.out, nullptr, st, false, next_amax,
+      rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, nullptr, L.bias, L.out, nullptr, st, false, out_word,
                        0, 0, true);
-      if (rc) return rc;
-      continue;
+      next_cleared = false;
+    } else {
+      const bool fed = i > 0 && feeds_next(layers, n, i - 1);  // input maximum already accumulated
+      if (!fed) {
+        const int64_t numel = pixels(L.shape) * L.shape.Cin;
+        rc = qvae_act_absmax(L.x, numel, in_word, st);
+        if (rc) return rc;
+      }
+      rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false, out_word,
+                       0, 0, false, in_word, x_scale, word[(i + 2) % 3]);
+      next_cleared = true;
     }
-    const int64_t numel = pixels(L.shape) * L.shape.Cin;
-    const bool fed = i > 0 && feeds_next(layers, n, i - 1);  // input absmax already accumulated
-    rc = fed ? launch_quant_from_amax(L.x, numel, amax_word[i & 1], xq, x_scale, next_amax, st)
-             : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, next_amax);
-    if (rc) return rc;
-    rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
-                     next_amax);
     if (rc) return rc;
   }
   return QVAE_OK;

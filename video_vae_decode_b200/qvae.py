@@ -32,7 +32,7 @@ EXPORTS = (
     "qvae_act_absmax", "qvae_act_quant_from_absmax",
     "qvae_causal_conv3d_w8a8_band", "qvae_causal_conv3d_w8a8_band_acc32",
     "qvae_packed_weight_bytes_bf16", "qvae_pack_weights_bf16", "qvae_causal_conv3d_bf16",
-    "qvae_causal_conv3d_bf16_acc32",
+    "qvae_causal_conv3d_bf16_acc32", "qvae_causal_conv3d_w8a8_fused", "qvae_causal_conv3d_w8a8_fused_acc32",
 )
 
 
@@ -87,6 +87,8 @@ def lib():
             "qvae_pack_weights_bf16": ([i32, i32, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_bf16": ([ctypes.POINTER(qvae_shape), p, p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_bf16_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_fused": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p, p], ctypes.c_int),
+            "qvae_causal_conv3d_w8a8_fused_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p, p], ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
             "qvae_decode_layers": ([ctypes.POINTER(qvae_layer), i32, p, sz, p], ctypes.c_int),
             "qvae_get_error": ([p], ctypes.c_int),
@@ -289,6 +291,38 @@ def qvae_causal_conv3d_w8a8_band_acc32(xq_band: torch.Tensor, halo_top: int, hal
     _check("qvae_causal_conv3d_w8a8_band_acc32",
            lib().qvae_causal_conv3d_w8a8_band_acc32(ctypes.byref(shp), int(halo_top), int(halo_bot),
                                                     _ptr(xq_band), _ptr(wq_packed), _ptr(acc), _stream(stream)))
+
+
+def qvae_causal_conv3d_w8a8_fused(x: torch.Tensor, x_amax: torch.Tensor, wq_packed: torch.Tensor,
+                                  w_scale: torch.Tensor, bias: Optional[torch.Tensor], out: torch.Tensor,
+                                  x_scale_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    """x bf16; x_amax a 4-byte device word from qvae_act_absmax (bf16 magnitude bits of max |x|)."""
+    shp = shape_of(x, int(out.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_fused",
+           lib().qvae_causal_conv3d_w8a8_fused(ctypes.byref(shp), _ptr(x), _ptr(x_amax), _ptr(wq_packed),
+                                               _ptr(w_scale), _ptr(bias), _ptr(out), _ptr(x_scale_out),
+                                               _stream(stream)))
+
+
+def qvae_causal_conv3d_w8a8_fused_acc32(x: torch.Tensor, x_amax: torch.Tensor, wq_packed: torch.Tensor,
+                                        acc: torch.Tensor, stream=None) -> None:
+    shp = shape_of(x, int(acc.shape[-1]))
+    _check("qvae_causal_conv3d_w8a8_fused_acc32",
+           lib().qvae_causal_conv3d_w8a8_fused_acc32(ctypes.byref(shp), _ptr(x), _ptr(x_amax), _ptr(wq_packed),
+                                                     _ptr(acc), _stream(stream)))
+
+
+def layer_w8a8(x, wq_packed, w_scale, bias, Cout: int, stream=None, amax=None, scale=None):
+    """One quantised layer the fused way: qvae_act_absmax, then the convolution quantising x itself.
+    Returns (out, scale)."""
+    if amax is None:
+        amax = torch.empty(1, dtype=torch.int32, device=x.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    out = torch.empty(tuple(x.shape[:-1]) + (Cout,), dtype=torch.bfloat16, device=x.device)
+    qvae_act_absmax(x, amax, stream)
+    qvae_causal_conv3d_w8a8_fused(x, amax, wq_packed, w_scale, bias, out, scale, stream)
+    return out, scale
 
 
 def conv_acc32(xq, wq_packed, Cout: int, stream=None):
