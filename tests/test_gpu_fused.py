@@ -69,7 +69,7 @@ def check(q, shape, seed, tiling=None, ctas=0, outliers=True, drift=False):
 
 TILINGS = [None, dict(mode=1), dict(mode=2), dict(mode=1, MS=1), dict(mode=2, MS=1), dict(mode=1, MS=3, G=1),
            dict(mode=2, MS=4, G=1), dict(mode=2, MS=2, NT=32), dict(mode=1, MS=2, SA=1, SB=2),
-           dict(mode=2, MS=2, NT=192, G=3, SA=2, SB=2)]
+           dict(mode=2, MS=2, NT=64, G=3, SA=2, SB=2)]
 
 
 @pytest.mark.parametrize("tiling", TILINGS)
