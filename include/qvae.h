@@ -387,8 +387,11 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
 int qvae_set_conv_cta_limit(int32_t max_ctas);
 
 /* The tiling the next convolution of this shape would use: out[0..7] = MS,
- * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G. */
-int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out8);
+ * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G.
+ * variant: 0 the W8A8 convolution of INT8 codes, 1 the fused W8A8
+ * convolution (bf16 input quantised in the kernel), 2 the native-precision
+ * convolution. */
+int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8);
 
 #if defined(__GNUC__)
 #pragma GCC visibility pop

@@ -136,14 +136,15 @@ def test_tiling_choice_is_valid():
         qvae.qvae_set_conv_tiling(MS=3, G=3)
 
 
-def test_tiling_choice_is_valid_over_the_supported_shapes():
-    """The cost model picks a launchable tiling for every shape the kernel accepts."""
+@pytest.mark.parametrize("variant", [0, 1, 2], ids=["codes", "fused", "native"])
+def test_tiling_choice_is_valid_over_the_supported_shapes(variant):
+    """The cost model picks a launchable tiling for every shape each kernel accepts."""
     chans = (32, 64, 96, 128, 160, 192, 256, 384, 512)
     for Cin in chans:
         for Cout in chans:
             for H, W in ((1, 1), (7, 33), (16, 8), (33, 7), (128, 128), (517, 300)):
                 for T in (1, 3):
-                    t = qvae.qvae_get_conv_tiling(1, T, H, W, Cin, Cout)
+                    t = qvae.qvae_get_conv_tiling(1, T, H, W, Cin, Cout, variant)
                     assert 1 <= t["MS"] <= 4 and t["MS"] * t["NT"] <= 512 and t["mode"] in (1, 2)
                     assert Cout % t["NT"] == 0 and t["NT"] % 32 == 0 and t["NT"] <= 256
                     assert 1 <= t["SA"] <= 12 and 1 <= t["SB"] <= 12

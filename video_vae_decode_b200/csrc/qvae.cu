@@ -950,15 +950,17 @@ int qvae_set_conv_cta_limit(int32_t max_ctas) {
   return QVAE_OK;
 }
 
-int qvae_get_conv_tiling(const qvae_shape* shape, int32_t* out8) {
-  if (!out8) return QVAE_ERR_ARG;
+int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8) {
+  if (!out8 || variant < 0 || variant > 2) return QVAE_ERR_ARG;
   int rc = check_shape(shape);
   if (rc) return rc;
   int sms = 148, dev;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) sm_count(dev, &sms);
   cudaGetLastError();
+  qvae_shape sb = *shape;
+  if (variant == 2) sb.Cin *= 2;  // native precision: tiled by bytes
   Tiling t;
-  if ((rc = make_tiling(*shape, &t, sms))) return rc;
+  if ((rc = make_tiling(sb, &t, sms, variant == 1))) return rc;
   out8[0] = t.MS;
   out8[1] = t.NT;
   out8[2] = t.SA;

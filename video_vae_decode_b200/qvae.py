@@ -96,7 +96,7 @@ def lib():
             "qvae_selftest_wait_timeout": ([u64, p], ctypes.c_int),
             "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
             "qvae_set_conv_cta_limit": ([i32], ctypes.c_int),
-            "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), ctypes.POINTER(i32)], ctypes.c_int),
+            "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), i32, ctypes.POINTER(i32)], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -434,8 +434,9 @@ def qvae_set_conv_cta_limit(max_ctas: int = 0) -> None:
     _check("qvae_set_conv_cta_limit", lib().qvae_set_conv_cta_limit(int(max_ctas)))
 
 
-def qvae_get_conv_tiling(N, T, H, W, Cin, Cout) -> dict:
+def qvae_get_conv_tiling(N, T, H, W, Cin, Cout, variant: int = 0) -> dict:
+    """variant 0: convolution of INT8 codes; 1: fused (bf16 input quantised in the kernel); 2: native bf16."""
     shp = make_shape(N, T, H, W, Cin, Cout)
     out = (ctypes.c_int32 * 8)()
-    _check("qvae_get_conv_tiling", lib().qvae_get_conv_tiling(ctypes.byref(shp), out))
+    _check("qvae_get_conv_tiling", lib().qvae_get_conv_tiling(ctypes.byref(shp), int(variant), out))
     return dict(zip(("MS", "NT", "SA", "SB", "acc_buffers", "ctas", "mode", "G"), list(out)))
