@@ -622,7 +622,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
                      : "r"(src + i * kStgPixelBytes + u * 32u + 16u));
-        const uint4 q = quant16(z, zero_scale, lo, hi);
+        const uint4 q = quant16_x2(z, zero_scale, lo, hi);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                          a_st + static_cast<uint32_t>(L) * 128u + ((static_cast<uint32_t>(u) ^ (L & 7u)) << 4)),
                      "r"(q.x), "r"(q.y), "r"(q.z), "r"(q.w)
@@ -715,7 +715,10 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       const uint32_t t_buf = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + accb * static_cast<uint32_t>(a.NT);
       for (int s = 0; s < a.MS && !dead; ++s) {
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(acc_full + 8 * (accb + s), cp, abort_flag, limit, kErrTimeoutEpilogue);
+        // in the fused variant the quantising warps share these warps' SM
+        // sub-partitions: poll with a back-off instead of spinning
+        if (lane == 0)
+          ok = mbar_wait(acc_full + 8 * (accb + s), cp, abort_flag, limit, kErrTimeoutEpilogue, kFuse ? 200u : 0u);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) {
           dead = true;

@@ -101,8 +101,10 @@ enum DeviceError : int {
 
 // Wait for the phase with the given parity to complete.  Returns false when
 // the CTA has been told to abort or when this wait ran past `limit_ns`.
+// backoff_ns > 0: sleep that long between polls, leaving the issue slots of
+// the SM sub-partition to warps that compute while this one waits.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t limit_ns, int err_code) {
+                                          uint64_t limit_ns, int err_code, uint32_t backoff_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -113,6 +115,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       atomicCAS(&g_qvae_error, 0, err_code);
       return false;
     }
+    if (backoff_ns) __nanosleep(backoff_ns);
   }
 }
 
