@@ -1,10 +1,11 @@
 """Benchmark of the W8A8 CausalConv3d layers of the VAE decoder on B200.
 
 One step = the whole per-call path of every layer of the workload: for each
-layer the activation absmax, then the implicit-GEMM convolution, which
-quantises its bf16 input to INT8 itself and applies the fused epilogue
-(weights are quantised and packed once, before timing, as a model load
-would).  Default workload: the six decoder
+layer the activation absmax + INT8 quantisation, then the implicit-GEMM
+convolution with its fused epilogue (weights are quantised and packed once,
+before timing, as a model load would).  --fused times the other form of a
+layer: the absmax pass, then the convolution that quantises its bf16 input
+itself.  Default workload: the six decoder
 layer shapes of a 1024x1024 decode (384->384 @128x128 and @256x256, 384->192
 and 192->192 @512x512, 192->96 and 96->96 @1024x1024, 1% outliers at +-8);
 its first layer is the same tensors as the single decoder top-stage layer
@@ -69,6 +70,8 @@ def parse():
                          "absmax, then per band quantise + band convolution)")
     ap.add_argument("--split", action="store_true",
                     help="split one image layer across the ranks by row bands (strong scaling)")
+    ap.add_argument("--fused", action="store_true",
+                    help="layers as absmax + the convolution quantising its bf16 input in the kernel")
     ap.add_argument("--chain", default="",
                     help="comma-separated consecutive layers of the workload run as one qvae_decode_layers "
                          "chain, each output feeding the next input (one GPU)")
@@ -351,6 +354,7 @@ class LayerJob:
             raise SystemExit("--bands and --chunk do not combine")
         self.starts = list(range(0, s.T, self.chunk)) if self.chunk else [0]
         self.dev = dev
+        self.fused = bool(args.fused) and not (self.chunk or self.nb)
 
     def set_bytes(self):
         s = self.s
@@ -396,14 +400,14 @@ class LayerJob:
     def launches_per_step(self):
         if self.nb:
             return 1 + 2 * self.nb
-        return 3 * len(self.starts) if self.chunk else 2   # plain: absmax + convolution
+        return 2 if self.fused else 3 * len(self.starts)  # fused: absmax + convolution
 
     def _parts(self, st):
         return st["chunks"] if self.chunk else [st]
 
     def act(self, st):
         q = self.qvae
-        if not self.nb and not self.chunk:
+        if self.fused:
             q.qvae_act_absmax(st["x"], st["amax"], self.stream)
             return
         if self.nb:
@@ -424,7 +428,7 @@ class LayerJob:
 
     def conv(self, st):
         q = self.qvae
-        if not self.nb and not self.chunk:
+        if self.fused:
             q.qvae_causal_conv3d_w8a8_fused(st["x"], st["amax"], st["packed"], self.s_w, self.b, st["out"],
                                             st["x_scale"], self.stream)
             return
@@ -438,7 +442,7 @@ class LayerJob:
 
     def step(self, st):
         q = self.qvae
-        if not self.nb and not self.chunk:
+        if self.fused:
             self.act(st)
             self.conv(st)
             return
@@ -587,11 +591,17 @@ def run_ours(args):
     scs = torch.empty(1, dtype=torch.float32, device=dev)
     outs = torch.empty((s0.N, s0.T, Hs, Ws, s0.Cout), dtype=torch.bfloat16, device=dev)
     switch_ms = []
+    xqs = torch.empty(xs.shape, dtype=torch.int8, device=dev)
+    wss = torch.empty(qvae.qvae_act_workspace_bytes(xs.numel()), dtype=torch.uint8, device=dev)
     for _ in range(2):                            # first call, then the same call warm
         torch.cuda.synchronize()
         t_sw = time.perf_counter()
-        qvae.qvae_act_absmax(xs, ams, stream)
-        qvae.qvae_causal_conv3d_w8a8_fused(xs, ams, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, scs, stream)
+        if jobs[0].fused:
+            qvae.qvae_act_absmax(xs, ams, stream)
+            qvae.qvae_causal_conv3d_w8a8_fused(xs, ams, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, scs, stream)
+        else:
+            qvae.qvae_act_absmax_quant(xs, xqs, scs, wss, stream)
+            qvae.qvae_causal_conv3d_w8a8(xqs, scs, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, stream)
         torch.cuda.synchronize()
         switch_ms.append((time.perf_counter() - t_sw) * 1e3)
     del xs, outs
@@ -664,9 +674,9 @@ def run_ours(args):
             "ms": p["layer"], "act_ms": p["act"], "conv_ms": p["conv"], "conv_ms_median": p["conv_median"],
             "layer_tops": lops / (p["layer"] * 1e-3) / 1e12, "conv_tops": lops / (p["conv"] * 1e-3) / 1e12,
             "conv_frac": lops / (p["conv"] * 1e-3) / 1e12 / peak,
-            "act_gbs": (2 if not (j.chunk or j.nb) else 5) * numel / (p["act"] * 1e-3) / 1e9,
+            "act_gbs": (2 if j.fused else 5) * numel / (p["act"] * 1e-3) / 1e9,
             "tiling": qvae.qvae_get_conv_tiling(j.s.N, j.s.T, j.s.H, j.s.W, j.s.Cin, j.s.Cout,
-                                                1 if not (j.chunk or j.nb) else 0),
+                                                1 if j.fused else 0),
             "dram_bytes_per_conv_launch": tr})
     traffic_mean = (sum(traffic) / len(traffic)) if all(t is not None for t in traffic) else None
     h2d = sum(j.layer.x.numel() * 2 for j in jobs)
@@ -679,8 +689,9 @@ def run_ours(args):
                    "arithmetic": ARITHMETIC,
                    "l2": (f"inputs, codes, outputs and packed weights rotate over {n_sets} buffer sets "
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
-                   "launch": ("one CUDA graph replay per step (per layer: act absmax, conv quantising in its "
-                              "producer)"
+                   "launch": (("one CUDA graph replay per step (per layer: act absmax, conv quantising in its "
+                               "producer)" if jobs[0].fused else
+                               "one CUDA graph replay per step (per layer: act absmax, act quantise, conv)")
                               if args.launch == "graph" else "direct launches from Python"),
                    "ops_per_step": ops,
                    "stream_chunk": (f"{jobs[0].chunk} frames, two carried" if jobs[0].chunk else None),
@@ -693,13 +704,14 @@ def run_ours(args):
                           "resolution_switch": {"shape": f"{Hs}x{Ws}", "first": switch_ms[0], "warm": switch_ms[1]},
                           "note": "host wall clock, act + conv of the first layer with a device synchronise"},
         "roofline": {"bound": "tensor", "achieved": conv_tops, "peak": peak, "unit": "TOPS",
-                     "kernel_variant": "conv3d_w8a8_fused_kernel (bf16 in, codes made in shared memory)",
+                     "kernel_variant": ("conv3d_w8a8_fused_kernel (bf16 in, codes made in shared memory)"
+                                        if jobs[0].fused else "conv3d_w8a8_kernel (INT8 codes in)"),
                      "frac": conv_tops / peak, "traffic": traffic_mean,
                      "peak_source": f"{peak_src} bf16 burst {bf16_burst} TFLOP/s x {INT8_PER_BF16} "
                                     "(nominal dense INT8/BF16 ratio)",
                      "int8_cublas_tops": int8_tops,
                      "frac_of_int8_cublas": (conv_tops / int8_tops) if int8_tops else None,
-                     "kernel": "conv3d_w8a8_fused_kernel",
+                     "kernel": "conv3d_w8a8_fused_kernel" if jobs[0].fused else "conv3d_w8a8_kernel",
                      "kernel_ms_mean": conv_total_max / len(jobs), "launches": conv_launches * len(jobs),
                      "note": ("achieved = the layers' ops over the sum of their convolutions' mean CUDA-event "
                               "times; traffic = mean DRAM bytes per conv launch over the layers")},

@@ -324,15 +324,20 @@ typedef struct qvae_layer {
   const void* bias;          /* bf16 [Cout] or NULL */
 } qvae_layer;
 
-/* Workspace bytes qvae_decode_layers needs (256): the last quantised layer's
- * activation scale (fp32 at byte 0) and three maximum words. */
+/* Workspace bytes qvae_decode_layers needs for these layers under the
+ * current qvae_set_fused_quant setting: the last quantised layer's activation
+ * scale (fp32 at byte 0) and three maximum words (bytes 64, 128, 192); with
+ * the two-pass path also the activation workspace and the largest quantised
+ * input's codes. */
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
 
 /*
- * In order on one stream, for each quantised layer: the activation absmax
- * into a workspace word, then the fused W8A8 convolution (which quantises x
- * itself) into `out`; for each native layer with packed bf16 weights: the
- * bf16 convolution into `out`; native layers without weights are skipped.
+ * In order on one stream, for each quantised layer: the activation absmax +
+ * quantise passes into the workspace, then the W8A8 convolution into `out`
+ * (with qvae_set_fused_quant(1): the absmax into a workspace word, then the
+ * fused convolution, which quantises x itself); for each native layer with
+ * packed bf16 weights: the bf16 convolution into `out`; native layers without
+ * weights are skipped.
  * All layers are validated before anything is launched.  When a layer's
  * `out` is the next layer's `x` and the next layer is quantised (same N, T,
  * H, W and Cout == next Cin), the convolution also accumulates the maximum
@@ -385,6 +390,15 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
  * A small cap makes each CTA walk several tiles of a small problem.
  */
 int qvae_set_conv_cta_limit(int32_t max_ctas);
+
+/*
+ * How qvae_decode_layers runs quantised layers (process-wide, tuning and
+ * tests): 0 (default) the quantise pass writes codes that the convolution
+ * reads; 1 the fused convolution quantises in its producer.  Both give the
+ * same codes, scales and outputs; the default is the one that measured
+ * faster on B200.  Query qvae_decode_workspace_bytes after changing it.
+ */
+int qvae_set_fused_quant(int32_t on);
 
 /* The tiling the next convolution of this shape would use: out[0..7] = MS,
  * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G.

@@ -806,12 +806,21 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
 }
 
 // Workspace of qvae_decode_layers: the activation scale of the last quantised
-// layer (fp32 at byte 0) and three 32-bit maximum words (bytes 64, 128, 192).
-constexpr size_t kDecodeWorkspace = 256;
+// layer (fp32 at byte 0) and three 32-bit maximum words (bytes 64, 128, 192);
+// then, when quantised layers run as the quantise pass + the convolution of
+// codes, the activation workspace (partial maxima) and the largest quantised
+// input's codes.
+constexpr size_t kDecodeHeader = 256;
+
+std::atomic<bool> g_fused_quant{false};  // quantised layers of qvae_decode_layers: fused convolution
 
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {
   if (!layers || n < 0) return 0;
-  return kDecodeWorkspace;
+  if (g_fused_quant) return kDecodeHeader;
+  int64_t max_in = 0;
+  for (int32_t i = 0; i < n; ++i)
+    if (layers[i].quantized) max_in = std::max<int64_t>(max_in, pixels(layers[i].shape) * layers[i].shape.Cin);
+  return kDecodeHeader + kActWorkspace + static_cast<size_t>((max_in + 255) / 256 * 256);
 }
 
 // The library runs a layer when it is quantised, or when it is a native-
@@ -852,11 +861,14 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       qvae_shape sb = layers[i].shape;
       if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
-      if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0))) return rc;
+      if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0 && g_fused_quant))) return rc;
     }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* x_scale = reinterpret_cast<float*>(ws);
+  const bool fused = g_fused_quant.load();
+  void* partial = ws + kDecodeHeader;
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + kDecodeHeader + kActWorkspace);
   // Layer i reads its input maximum from word i % 3, accumulates its output's
   // maximum (when that output feeds the next quantised layer) into word
   // (i + 1) % 3, and a fused convolution clears word (i + 2) % 3: the word
@@ -876,7 +888,9 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
     const bool feeds = feeds_next(layers, n, i);
     uint32_t* in_word = word[i % 3];
     uint32_t* out_word = feeds ? word[(i + 1) % 3] : nullptr;
-    if (out_word && !next_cleared) QVAE_CUDA(cudaMemsetAsync(out_word, 0, sizeof(uint32_t), st));
+    // the quantise pass of the two-pass path clears out_word itself
+    if (out_word && !next_cleared && (fused || !L.quantized))
+      QVAE_CUDA(cudaMemsetAsync(out_word, 0, sizeof(uint32_t), st));
     int rc;
     if (!L.quantized) {
       // native precision: the bf16 convolution straight from the bf16 input
@@ -885,14 +899,21 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       next_cleared = false;
     } else {
       const bool fed = i > 0 && feeds_next(layers, n, i - 1);  // input maximum already accumulated
-      if (!fed) {
-        const int64_t numel = pixels(L.shape) * L.shape.Cin;
-        rc = qvae_act_absmax(L.x, numel, in_word, st);
+      const int64_t numel = pixels(L.shape) * L.shape.Cin;
+      if (fused) {
+        if (!fed && (rc = qvae_act_absmax(L.x, numel, in_word, st))) return rc;
+        rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
+                         out_word, 0, 0, false, in_word, x_scale, word[(i + 2) % 3]);
+        next_cleared = true;
+      } else {
+        // quantise pass (which also clears out_word), then the convolution of the codes
+        rc = fed ? launch_quant_from_amax(L.x, numel, in_word, xq, x_scale, out_word, st)
+                 : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, out_word);
         if (rc) return rc;
+        rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
+                         out_word);
+        next_cleared = false;
       }
-      rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false, out_word,
-                       0, 0, false, in_word, x_scale, word[(i + 2) % 3]);
-      next_cleared = true;
     }
     if (rc) return rc;
   }
@@ -941,6 +962,12 @@ int qvae_set_conv_tiling(int32_t MS, int32_t NT, int32_t SA, int32_t SB, int32_t
   g_force[3] = SB;
   g_force[4] = mode;
   g_force[5] = G;
+  return QVAE_OK;
+}
+
+int qvae_set_fused_quant(int32_t on) {
+  if (on < 0 || on > 1) return QVAE_ERR_ARG;
+  g_fused_quant = on != 0;
   return QVAE_OK;
 }
 

@@ -33,6 +33,7 @@ EXPORTS = (
     "qvae_causal_conv3d_w8a8_band", "qvae_causal_conv3d_w8a8_band_acc32",
     "qvae_packed_weight_bytes_bf16", "qvae_pack_weights_bf16", "qvae_causal_conv3d_bf16",
     "qvae_causal_conv3d_bf16_acc32", "qvae_causal_conv3d_w8a8_fused", "qvae_causal_conv3d_w8a8_fused_acc32",
+    "qvae_set_fused_quant",
 )
 
 
@@ -96,6 +97,7 @@ def lib():
             "qvae_selftest_wait_timeout": ([u64, p], ctypes.c_int),
             "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
             "qvae_set_conv_cta_limit": ([i32], ctypes.c_int),
+            "qvae_set_fused_quant": ([i32], ctypes.c_int),
             "qvae_get_conv_tiling": ([ctypes.POINTER(qvae_shape), i32, ctypes.POINTER(i32)], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -428,6 +430,10 @@ def qvae_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
 
 def qvae_set_conv_tiling(MS=0, NT=0, SA=0, SB=0, mode=0, G=0) -> None:
     _check("qvae_set_conv_tiling", lib().qvae_set_conv_tiling(MS, NT, SA, SB, mode, G))
+
+
+def qvae_set_fused_quant(on: int = 0) -> None:
+    _check("qvae_set_fused_quant", lib().qvae_set_fused_quant(int(on)))
 
 
 def qvae_set_conv_cta_limit(max_ctas: int = 0) -> None:
