@@ -111,6 +111,7 @@ struct ConvArgs {
   int stg_groups;             // staging slots per activation box: (16 * MS + 2) / stg_rows
   uint32_t stg_slot_bytes;    // stg_rows x 10 pixels x 128 channels x 2 bytes
   uint32_t* zero_word;        // or null: a word set to zero (for a later layer's maximum)
+  float one;                  // 1.0f (an operand the compiler cannot fold; see add_f32x2)
 };
 
 constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
@@ -122,6 +123,23 @@ constexpr int kMaxStgSlots = 8;
 constexpr uint32_t kStgPixelBytes = 256;            // 128 bf16 channels of one pixel
 constexpr uint32_t kEpiBufBytes = 2048;    // one epilogue staging buffer: 32 pixels x 64 B
 constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
+
+// Packed fp32 pairs (low word = first value).  RN(a * b); and RN(a + b)
+// computed as fma(a, one, b) with `one` = (1.0, 1.0) from a kernel argument:
+// the assembler contracts a packed multiply followed by a packed add into one
+// fused multiply-add even with explicit round-to-nearest (one rounding where
+// the epilogue needs two), and it cannot fold a multiplier whose value it
+// does not know.
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t one, uint64_t b) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(one), "l"(b));
+  return r;
+}
 
 struct TileCoord {
   int n, t, h0, w0, co0;
@@ -357,8 +375,9 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 8 * kAccBars;
-  const uint32_t stg_full = acc_empty + 8 * kAccBars, stg_empty = stg_full + 8 * kMaxStgSlots;
-  const uint32_t drain_bar = stg_empty + 8 * kMaxStgSlots;
+  // stg_done: per staging slot, a running count of quantising-warp passes over it (a plain word, 8 bytes apart)
+  const uint32_t stg_full = acc_empty + 8 * kAccBars, stg_done = stg_full + 8 * kMaxStgSlots;
+  const uint32_t drain_bar = stg_done + 8 * kMaxStgSlots;
   uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
   volatile uint32_t* const tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -386,7 +405,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     if (kFuse) {
       for (int i = 0; i < a.SS; ++i) {
         mbar_init(stg_full + 8 * i, 1);
-        mbar_init(stg_empty + 8 * i, kCvtWarps);
+        asm volatile("st.shared.u32 [%0], 0;" ::"r"(stg_done + 8 * i) : "memory");
       }
     }
     for (int i = 0; i < a.SB; ++i) {
@@ -538,15 +557,17 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     // The activation boxes of the fused variant, in the MMA's order: each
     // box (tile, temporal tap, 128-channel chunk) is 16*MS + 2 rows x 10
     // columns of bf16 pixels, brought in as row groups of stg_rows rows by
-    // TMA into the staging ring (lane 0 of the first quantising warp keeps
-    // SS groups in flight) and turned into codes, 16 channels per item, in
+    // TMA into the staging ring (SS groups in flight) and turned into codes in
     // the 128-byte-swizzled K-major layout of the activation ring.  Rows and
     // columns beyond the image arrive as zeros from the tensor map and give
-    // code 0.  When a box is complete, each warp fences its shared-memory
-    // writes for the tensor cores and arrives on the (leader's) a_full.
+    // code 0.  Each lane converts one 16-byte piece (8 channels) of a pixel
+    // (consecutive lanes read consecutive pieces: no bank conflicts); lanes
+    // 2k and 2k + 1 hold one 16-channel group and the even one stores it.
+    // The warp that finishes a staging slot last refills it with the group SS
+    // positions ahead.  When a box is complete each warp fences its shared-
+    // memory writes for the tensor cores and arrives on the (leader's) a_full.
     const int cw = warp - (2 + kEpiWarps);
     const int ct = cw * 32 + lane;
-    const bool pf_thread = cw == 0 && lane == 0;
     struct Pos {
       int tile, kb, g, nkb, kt_lo;
       TileCoord c;
@@ -567,8 +588,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       if (++p.kb < p.nkb) return;
       start(p, p.tile + tile_step);
     };
-    uint32_t stg_armed = 0, stg_par = 0;
-    // issue the TMA load of position p into staging slot `slot` (use parity `par`)
+    // the TMA load of position p into staging slot `slot`
     auto issue = [&](const Pos& p, uint32_t slot) {
       const int kt = p.kt_lo + p.kb / a.nchunks, ch = p.kb % a.nchunks;
       const int frame = p.c.t + kt - 2 + 2 * a.carry;
@@ -588,64 +608,80 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     Pos cur, pf;
     start(cur, first_tile);
     start(pf, first_tile);
-    if (pf_thread) {
-      for (uint32_t k = 0; k < static_cast<uint32_t>(a.SS) && pf.tile < a.num_tiles; ++k) {
+    uint32_t stg_armed = 0, stg_par = 0;  // (lane 0 of the issuing warp) slots with a load in flight
+    for (uint32_t k = 0; k < static_cast<uint32_t>(a.SS) && pf.tile < a.num_tiles; ++k) {
+      if (ct == 0) {
         issue(pf, k);
         stg_armed |= 1u << k;
-        advance(pf);
       }
+      advance(pf);
     }
     uint32_t slot = 0, sp = 0, as = 0, ap = 0;
     const int lines = a.stg_rows * kBoxW;
     bool ok = true;
-    while (ok && cur.tile < a.num_tiles) {
+    // 8 bf16 values -> 8 codes (two words)
+    auto codes8 = [&](const uint4& v) -> uint2 {
+      if (zero_scale) return make_uint2(0u, 0u);
+      if (z.exact) return make_uint2(quant4(z, v.x, v.y), quant4(z, v.z, v.w));
+      return make_uint2(quant4_x2(z, v.x, v.y), quant4_x2(z, v.z, v.w));
+    };
+    while (cur.tile < a.num_tiles) {
       const int ch = cur.kb % a.nchunks;
-      const int nu = (ch == a.nchunks - 1) ? 2 * a.last_ksteps : 8;  // 16-channel groups the MMA reads
+      const int np = (ch == a.nchunks - 1) ? 4 * a.last_ksteps : 16;  // 8-channel pieces the MMA reads
       const uint32_t a_st = a_ring + as * a.a_stage_bytes;
-      // every lane waits (so that each observes the copies it reads); the
-      // warp leaves together if any lane's wait gave up
-      bool waited = cur.g != 0 || mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutConvert);
-      waited = waited && mbar_wait(stg_full + 8 * slot, sp, abort_flag, limit, kErrTimeoutConvert);
-      if (!__all_sync(0xFFFFFFFFu, waited)) {
+      int waited = 1;
+      if (lane == 0) {
+        if (cur.g == 0) waited = mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutConvert);
+        if (waited) waited = mbar_wait(stg_full + 8 * slot, sp, abort_flag, limit, kErrTimeoutConvert);
+      }
+      if (!__shfl_sync(0xFFFFFFFFu, waited, 0)) {
         ok = false;
         break;
       }
+      __syncwarp();  // lane 0's acquire covers the whole warp's accesses
       const uint32_t src = stg_ring + slot * a.stg_slot_bytes;
       const int line0 = cur.g * lines;
-      for (int it = ct; it < lines * nu; it += 32 * kCvtWarps) {
-        const int i = it / nu, u = it - i * nu;
-        const int L = line0 + i;
-        uint4 lo, hi;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w)
-                     : "r"(src + i * kStgPixelBytes + u * 32u));
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
-                     : "r"(src + i * kStgPixelBytes + u * 32u + 16u));
-        const uint4 q = quant16_x2(z, zero_scale, lo, hi);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         a_st + static_cast<uint32_t>(L) * 128u + ((static_cast<uint32_t>(u) ^ (L & 7u)) << 4)),
-                     "r"(q.x), "r"(q.y), "r"(q.z), "r"(q.w)
-                     : "memory");
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(stg_empty + 8 * slot);
-      if (pf_thread) {
-        // refill this slot with the group SS positions ahead, once both warps are done with it
-        if (pf.tile < a.num_tiles) {
-          if (!mbar_wait(stg_empty + 8 * slot, sp, abort_flag, limit, kErrTimeoutConvert)) {
-            stg_armed &= ~(1u << slot);
-            ok = false;
-          } else {
-            issue(pf, slot);
-            stg_par = (stg_par & ~(1u << slot)) | ((sp ^ 1u) << slot);
-            advance(pf);
-          }
-        } else {
-          stg_armed &= ~(1u << slot);
+      const int total = lines * np;
+      for (int base = 0; base < total; base += 32 * kCvtWarps) {
+        const int idx = base + ct;
+        const bool valid = idx < total;
+        const int i = idx / np, p = idx - i * np;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (valid)
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(src + static_cast<uint32_t>(i) * kStgPixelBytes + static_cast<uint32_t>(p) * 16u));
+        const uint2 c = codes8(v);
+        const uint32_t ox = __shfl_xor_sync(0xFFFFFFFFu, c.x, 1), oy = __shfl_xor_sync(0xFFFFFFFFu, c.y, 1);
+        if (valid && (p & 1) == 0) {
+          const uint32_t L = static_cast<uint32_t>(line0 + i), u = static_cast<uint32_t>(p >> 1);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_st + L * 128u + ((u ^ (L & 7u)) << 4)),
+                       "r"(c.x), "r"(c.y), "r"(ox), "r"(oy)
+                       : "memory");
         }
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      __syncwarp();
+      if (lane == 0) {
+        // the last warp done with this slot's current load refills it (the other warps' reads are ordered before)
+        uint32_t prev;
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "r"(stg_done + 8 * slot)
+                     : "memory");
+        if (prev % kCvtWarps == kCvtWarps - 1) {
+          fence_proxy_async_smem();
+          if (pf.tile < a.num_tiles) {
+            issue(pf, slot);
+            stg_armed |= 1u << slot;
+            stg_par = (stg_par & ~(1u << slot)) | ((sp ^ 1u) << slot);
+          } else {
+            stg_armed &= ~(1u << slot);
+          }
+        } else {
+          stg_armed &= ~(1u << slot);  // the other warp owns the refill
+        }
+      }
+      advance(pf);
       if (++slot == static_cast<uint32_t>(a.SS)) { slot = 0; sp ^= 1; }
       if (cur.g == a.stg_groups - 1) {
         // the box is complete: make the codes visible to the tensor cores
@@ -662,12 +698,13 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       }
       advance(cur);
     }
-    if (pf_thread && *abort_flag) {
-      // let the staging loads still in flight land before the CTA exits
+    if (lane == 0 && *abort_flag) {
+      // let the staging loads this warp issued and that are still in flight land before the CTA exits
       int dummy = 0;
       for (int i = 0; i < a.SS; ++i)
         if (stg_armed >> i & 1) mbar_wait(stg_full + 8 * i, stg_par >> i & 1, &dummy, limit, kErrTimeoutDrain);
     }
+    (void)ok;
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // A warp may read only the TMEM lane quarter warp % 4; lane quarter q holds
@@ -741,32 +778,27 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
                                    static_cast<int>(v[4 * e + 2]), static_cast<int>(v[4 * e + 3]));
             }
           } else {
-            const float4* sc4 = reinterpret_cast<const float4*>(sc + cc);
-            const float4* bi4 = reinterpret_cast<const float4*>(bi + cc);
+            // scale and bias pairs (channels 2i, 2i + 1) as packed fp32
+            const uint64_t one2 = (static_cast<uint64_t>(__float_as_uint(a.one)) << 32) | __float_as_uint(a.one);
+            const uint64_t* sc2 = reinterpret_cast<const uint64_t*>(sc + cc);
+            const uint64_t* bi2 = reinterpret_cast<const uint64_t*>(bi + cc);
             uint32_t packed[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              // y = float(acc) * scale, rounded, then + bias, rounded.  The
-              // scalar _rn intrinsics are never contracted into an FMA (packed
-              // f32x2 multiply + add were: one rounding instead of two).
-              const float4 b = bi4[e];
-              float y0, y1, y2, y3;
+            for (int e = 0; e < 16; ++e) {
+              // two channels at a time on the packed fp32 pipe:
+              // y = float(acc) * scale, rounded, then + bias, rounded (the
+              // explicit .rn forms are never contracted into an FMA)
+              uint64_t y;
               if (kBf16) {  // fp32 accumulators: y = acc + bias
-                y0 = __fadd_rn(__uint_as_float(v[4 * e]), b.x);
-                y1 = __fadd_rn(__uint_as_float(v[4 * e + 1]), b.y);
-                y2 = __fadd_rn(__uint_as_float(v[4 * e + 2]), b.z);
-                y3 = __fadd_rn(__uint_as_float(v[4 * e + 3]), b.w);
+                y = add_f32x2((static_cast<uint64_t>(v[2 * e + 1]) << 32) | v[2 * e], one2, bi2[e]);
               } else {
-                const float4 f = sc4[e];
-                y0 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e])), f.x), b.x);
-                y1 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 1])), f.y), b.y);
-                y2 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 2])), f.z), b.z);
-                y3 = __fadd_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[4 * e + 3])), f.w), b.w);
+                const uint64_t f = (static_cast<uint64_t>(__float_as_uint(__int2float_rn(static_cast<int>(v[2 * e + 1])))) << 32) |
+                                   __float_as_uint(__int2float_rn(static_cast<int>(v[2 * e])));
+                y = add_f32x2(mul_f32x2(f, sc2[e]), one2, bi2[e]);
               }
-              const __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
-              const __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
-              packed[2 * e] = *reinterpret_cast<const uint32_t*>(&p0);
-              packed[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+              const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(static_cast<uint32_t>(y)),
+                                                              __uint_as_float(static_cast<uint32_t>(y >> 32)));
+              packed[e] = *reinterpret_cast<const uint32_t*>(&p2);
             }
             if (a.out_amax) {
               // the next layer's activation absmax, taken on what is written
@@ -824,7 +856,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         __syncwarp();
         if (lane == 0) {
           if (kPair) {
-            mbar_arrive_cluster(empty_leader + 8 * (accb + s));
+            mbar_arrive_remote(empty_leader + 8 * (accb + s));
           } else {
             mbar_arrive(acc_empty + 8 * (accb + s));
           }

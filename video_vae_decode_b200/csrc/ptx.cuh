@@ -276,6 +276,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Arrive on a barrier of another CTA of the cluster with release at CTA
+// scope only: for a signal that follows completed work of this thread (TMEM
+// reads finished by tcgen05.wait::ld), which needs no cluster-wide ordering
+// of this thread's earlier writes -- a cluster-scope release also waits for
+// them, e.g. for a bulk store just issued.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tc_fence_before() {

@@ -432,6 +432,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   a.x_amax = x_amax;
   a.x_scale_out = x_scale_out;
   a.zero_word = zero_word;
+  a.one = 1.0f;
   a.SS = t.SS;
   a.stg_rows = kStgRows;
   a.stg_groups = (t.MS * qvae::kTileRows + 2) / kStgRows;
