@@ -173,12 +173,47 @@ struct MmaRings {
   uint32_t tmem_base;
 };
 
-// MMA issuer (one thread of the pair's leader CTA).  Descriptors are built
-// once; every operand start inside the rings is the base descriptor plus an
-// offset in 16-byte units (all offsets stay inside the 14-bit start-address
-// field), so each MMA costs a few integer adds.  A weight stage holds kG
-// taps; per tap: kMS sub-tiles, each four k-steps of 32 channels into its own
-// accumulator.  One wait and one commit per stage.
+// One lane of a converged warp (the lowest active one).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
+template <int N>
+using IntC = std::integral_constant<int, N>;
+
+// Calls f(IntC<k>{}) for the run-time k-step count k (1 to 4), so that the
+// MMA sequence of a stage is straight-line code for every chunk width.
+template <typename F>
+__device__ __forceinline__ void with_ksteps(uint32_t ksteps, F&& f) {
+  switch (ksteps) {
+    case 4:
+      f(IntC<4>{});
+      break;
+    case 3:
+      f(IntC<3>{});
+      break;
+    case 2:
+      f(IntC<2>{});
+      break;
+    default:
+      f(IntC<1>{});
+      break;
+  }
+}
+
+// MMA issuer: the whole warp 1 of the pair's leader CTA runs the loop, so
+// that the descriptor arithmetic is warp-uniform, and one elected lane issues
+// each tcgen05 instruction; lane 0 waits on the barriers and broadcasts the
+// outcome.  (Issued by a lone thread, the same MMAs measured up to twice the
+// tensor pipe's cycles each at N = 96.)  Descriptors are built once; every
+// operand start inside the rings is the base descriptor plus an offset in
+// 16-byte units (all offsets stay inside the 14-bit start-address field).  A
+// weight stage holds kG taps; per tap: kMS sub-tiles, each k-steps of 32
+// bytes of K into its own accumulator.  One wait and one commit per stage.
 //
 // Accumulator barriers are per (buffer, sub-tile).  With a single buffer
 // (split mode) the first and the last 128-channel chunk of a tile are issued
@@ -191,6 +226,7 @@ template <bool kBf16, bool kPair, bool kFuse, int kMS, int kG>
 __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings& r,
                                                volatile int* abort_flag, uint64_t limit, int first_tile,
                                                int tile_step, uint32_t rank, bool& issued) {
+  const int lane = static_cast<int>(threadIdx.x & 31);
   const uint32_t idesc = kBf16 ? idesc_bf16(kPair ? 256 : 128, a.NT) : idesc_i8(kPair ? 256 : 128, a.NT);
   const uint64_t a_desc0 = sw128_kmajor_desc(r.a_ring, kGroupStride);
   const uint64_t b_desc0 = sw128_kmajor_desc(r.b_ring, 1024u);
@@ -203,34 +239,39 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   const bool split = a.split != 0;
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
   bool b_ready = false;  // b_full of stage bs already seen complete
+  // lane 0 waits; the warp takes its outcome
+  auto wait = [&](uint32_t bar, uint32_t parity, bool cluster_scope) -> bool {
+    int ok = 1;
+    if (lane == 0) {
+      ok = cluster_scope ? mbar_wait_cluster(bar, parity, abort_flag, limit, kErrTimeoutMma)
+                         : mbar_wait(bar, parity, abort_flag, limit, kErrTimeoutMma);
+    }
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+  };
   auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
-    if (kBf16) {
-      if (kPair) {
-        mma_bf16_pair(d, ad, bd, idesc, acc);
+    if (elect_one()) {
+      if (kBf16) {
+        if (kPair) {
+          mma_bf16_pair(d, ad, bd, idesc, acc);
+        } else {
+          mma_bf16(d, ad, bd, idesc, acc);
+        }
+      } else if (kPair) {
+        mma_i8_pair(d, ad, bd, idesc, acc);
       } else {
-        mma_bf16(d, ad, bd, idesc, acc);
+        mma_i8(d, ad, bd, idesc, acc);
       }
-    } else if (kPair) {
-      mma_i8_pair(d, ad, bd, idesc, acc);
-    } else {
-      mma_i8(d, ad, bd, idesc, acc);
     }
   };
   auto commit = [&](uint32_t bar) {
-    if (kPair) {
-      mma_commit_pair_multicast(bar, 0x3);
-    } else {
-      mma_commit(bar);
-    }
-  };
-  // the MMAs of one tap for sub-tile s
-  auto tap_mmas = [&](uint32_t d, uint64_t a_tap, uint64_t b_tap, uint32_t ksteps, uint32_t acc) {
-    if (ksteps == 4u) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
-        mma(d, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
-    } else {
-      for (uint32_t k = 0; k < ksteps; ++k) mma(d, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+    if (elect_one()) {
+      if (kPair) {
+        mma_commit_pair_multicast(bar, 0x3);
+      } else {
+        mma_commit(bar);
+      }
     }
   };
   for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
@@ -242,18 +283,14 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
     if (!split) {
 #pragma unroll
       for (int s = 0; s < kMS; ++s)
-        if (!mbar_wait(r.acc_empty + 8 * (accb + s), cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
+        if (!wait(r.acc_empty + 8 * (accb + s), cp ^ 1, false)) return false;
       tc_fence_after();
     }
     uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
     for (int kb = 0; kb < nkb; ++kb) {
       const int ch = kb % a.nchunks;
       // the fused variant's A stages are written by threads of both CTAs of a pair
-      if (kFuse && kPair) {
-        if (!mbar_wait_cluster(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) return false;
-      } else if (!mbar_wait(r.a_full + 8 * as, ap, abort_flag, limit, kErrTimeoutMma)) {
-        return false;
-      }
+      if (!wait(r.a_full + 8 * as, ap, kFuse && kPair)) return false;
       tc_fence_after();
       const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
       const uint64_t a_stage = a_desc0 + as * a_stage16;
@@ -264,7 +301,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
 #pragma unroll
         for (int s = 0; s < kMS; ++s) {
           if (first) {
-            if (!mbar_wait(r.acc_empty + 8 * s, cp ^ 1, abort_flag, limit, kErrTimeoutMma)) return false;
+            if (!wait(r.acc_empty + 8 * s, cp ^ 1, false)) return false;
             tc_fence_after();
           }
           uint32_t acc_s = first ? 0u : 1u;
@@ -272,18 +309,24 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
           sp = bp;
           for (int grp = 0; grp < kGrp; ++grp) {
             if (s == 0) {
-              if (!mbar_wait(r.b_full + 8 * st, sp, abort_flag, limit, kErrTimeoutMma)) return false;
+              if (!wait(r.b_full + 8 * st, sp, false)) return false;
               tc_fence_after();
             }
             const uint64_t b_stage = b_desc0 + st * b_stage16;
+            with_ksteps(ksteps, [&](auto KS) {
+              constexpr int ks = decltype(KS)::value;
 #pragma unroll
-            for (int g = 0; g < kG; ++g) {
-              const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
-              const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
-              const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4) + s * sub16;
-              tap_mmas(d_tile + s * nt, a_tap, b_stage + g * b_tap16, ksteps, acc_s);
-              acc_s = 1u;
-            }
+              for (int g = 0; g < kG; ++g) {
+                const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+                const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+                const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4) + s * sub16;
+                const uint64_t b_tap = b_stage + g * b_tap16;
+#pragma unroll
+                for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
+                  mma(d_tile + s * nt, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc_s : 1u);
+                acc_s = 1u;
+              }
+            });
             issued = true;
             if (s == kMS - 1) commit(r.b_empty + 8 * st);
             if (++st == sb) { st = 0; sp ^= 1; }
@@ -296,39 +339,36 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
         acc = 1u;
       } else {
         for (int grp = 0; grp < kGrp; ++grp) {
-          if (!b_ready && !mbar_wait(r.b_full + 8 * bs, bp, abort_flag, limit, kErrTimeoutMma)) return false;
+          if (!b_ready && !wait(r.b_full + 8 * bs, bp, false)) return false;
           tc_fence_after();
           {
             // probe the next weight stage now; its result is used only after this
             // stage's MMAs are issued, so the probe's latency is hidden behind them
             const uint32_t nbs = (bs + 1 == sb) ? 0u : bs + 1;
             const uint32_t nbp = (bs + 1 == sb) ? bp ^ 1u : bp;
-            b_ready = mbar_test_wait(r.b_full + 8 * nbs, nbp);
+            int ready = 0;
+            if (lane == 0) ready = mbar_test_wait(r.b_full + 8 * nbs, nbp) ? 1 : 0;
+            b_ready = __shfl_sync(0xFFFFFFFFu, ready, 0) != 0;
           }
           const uint64_t b_stage = b_desc0 + bs * b_stage16;
+          with_ksteps(ksteps, [&](auto KS) {
+            constexpr int ks = decltype(KS)::value;
 #pragma unroll
-          for (int g = 0; g < kG; ++g) {
-            const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
-            const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
-            // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
-            const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
-            const uint64_t b_tap = b_stage + g * b_tap16;
-            if (ksteps == 4u) {
-#pragma unroll
-              for (int s = 0; s < kMS; ++s) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)  // 32 bytes of K = 2 units
-                  mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
-              }
-            } else {
+            for (int g = 0; g < kG; ++g) {
+              const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+              const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+              // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+              const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+              const uint64_t b_tap = b_stage + g * b_tap16;
 #pragma unroll
               for (int s = 0; s < kMS; ++s) {
-                for (uint32_t k = 0; k < ksteps; ++k)
+#pragma unroll
+                for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
                   mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
               }
+              acc = 1u;
             }
-            acc = 1u;
-          }
+          });
           issued = true;
           commit(r.b_empty + 8 * bs);
           if (++bs == sb) { bs = 0; bp ^= 1; }
@@ -509,7 +549,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       for (int i = 0; i < a.SB; ++i)
         if (b_armed >> i & 1) mbar_wait(b_full + 8 * i, b_par >> i & 1, &dummy, limit, kErrTimeoutDrain);
     }
-  } else if (warp == 1 && lane == 0 && leader) {
+  } else if (warp == 1 && leader) {
     // ---------------------------------------------------------- MMA issuer
     // One instantiation per (sub-tile count, taps per stage), so that the
     // MMA sequence of a stage is straight-line code.
@@ -542,7 +582,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         ok = run(std::integral_constant<int, 4>{}, G1{});
         break;
     }
-    if (!ok && *abort_flag && issued) {
+    if (!ok && issued && lane == 0 && *abort_flag) {
       // Wait for the tensor cores to finish what was issued before TMEM is freed.
       int dummy = 0;
       if (kPair) {
@@ -552,6 +592,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       }
       mbar_wait(drain_bar, 0, &dummy, limit, kErrTimeoutDrain);
     }
+    __syncwarp();
   } else if (kFuse && warp >= 2 + kEpiWarps) {
     // ----------------------------------------------------------- quantisers
     // The activation boxes of the fused variant, in the MMA's order: each
@@ -872,8 +913,8 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     }
   }
 
-  // Reconverge every warp (one lane of warps 0 and 1 ran a role alone) before
-  // the warp-aligned block / cluster barrier.
+  // Reconverge every warp (one lane of warp 0 ran a role alone) before the
+  // warp-aligned block / cluster barrier.
   __syncwarp();
   tc_fence_before();
   if (kPair) {
