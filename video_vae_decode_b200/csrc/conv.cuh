@@ -238,7 +238,23 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
   const uint32_t sb = static_cast<uint32_t>(a.SB);
   const bool split = a.split != 0;
   uint32_t as = 0, ap = 0, bs = 0, bp = 0, cs = 0, cp = 0;
-  bool b_ready = false;  // b_full of stage bs already seen complete
+  // phases already seen complete by a lookahead probe (a probe's result is
+  // read only after the MMAs issued behind it, so its latency stays hidden)
+  bool b_ready = false;    // b_full of stage bs
+  bool a_ready = false;    // a_full of stage as
+  bool acc_ready = false;  // the accumulator buffer of the next tile is free
+  const int tiles_per_frame = a.tiles_n * a.tiles_w * a.tiles_h;
+  // k-blocks (temporal tap x 128-channel chunk) of a tile: taps that meet the
+  // causal zero frames are skipped
+  auto tile_nkb = [&](int tile) -> int {
+    const int t = a.T == 1 ? 0 : (tile / tiles_per_frame) % a.T;
+    const int kt_lo = (a.carry || t >= 2) ? 0 : 2 - t;
+    return (3 - kt_lo) * a.nchunks;
+  };
+  auto probe = [&](uint32_t bar, uint32_t parity) -> int {
+    return lane == 0 ? (mbar_test_wait(bar, parity) ? 1 : 0) : 0;
+  };
+  auto seen = [&](int pr) -> bool { return __shfl_sync(0xFFFFFFFFu, pr, 0) != 0; };
   // lane 0 waits; the warp takes its outcome
   auto wait = [&](uint32_t bar, uint32_t parity, bool cluster_scope) -> bool {
     int ok = 1;
@@ -274,24 +290,25 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
       }
     }
   };
+  (void)rank;
   for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
-    const TileCoord c = decode_tile<kPair>(a, tile, rank);
-    const int kt_lo = (a.carry || c.t >= 2) ? 0 : 2 - c.t;  // taps that meet causal zero frames are skipped
-    const int nkb = (3 - kt_lo) * a.nchunks;
+    const int nkb = tile_nkb(tile);
     const uint32_t d_tile = r.tmem_base + cs * static_cast<uint32_t>(kMS) * nt;
     const uint32_t accb = cs * static_cast<uint32_t>(kMS);  // this buffer's first barrier index
     if (!split) {
-#pragma unroll
-      for (int s = 0; s < kMS; ++s)
-        if (!wait(r.acc_empty + 8 * (accb + s), cp ^ 1, false)) return false;
+      // the epilogue warps release a buffer's sub-tiles in order: the last one's
+      // barrier completing implies the others'
+      if (!acc_ready && !wait(r.acc_empty + 8 * (accb + kMS - 1), cp ^ 1, false)) return false;
       tc_fence_after();
     }
+    acc_ready = false;
     uint32_t acc = 0;  // the tile's first MMA overwrites the accumulator
     for (int kb = 0; kb < nkb; ++kb) {
       const int ch = kb % a.nchunks;
       // the fused variant's A stages are written by threads of both CTAs of a pair
-      if (!wait(r.a_full + 8 * as, ap, kFuse && kPair)) return false;
+      if (!a_ready && !wait(r.a_full + 8 * as, ap, kFuse && kPair)) return false;
       tc_fence_after();
+      a_ready = false;
       const uint32_t ksteps = (ch == a.nchunks - 1) ? static_cast<uint32_t>(a.last_ksteps) : 4u;
       const uint64_t a_stage = a_desc0 + as * a_stage16;
       const bool first = kb == 0, last = kb == nkb - 1;
@@ -341,14 +358,21 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
         for (int grp = 0; grp < kGrp; ++grp) {
           if (!b_ready && !wait(r.b_full + 8 * bs, bp, false)) return false;
           tc_fence_after();
-          {
-            // probe the next weight stage now; its result is used only after this
-            // stage's MMAs are issued, so the probe's latency is hidden behind them
-            const uint32_t nbs = (bs + 1 == sb) ? 0u : bs + 1;
-            const uint32_t nbp = (bs + 1 == sb) ? bp ^ 1u : bp;
-            int ready = 0;
-            if (lane == 0) ready = mbar_test_wait(r.b_full + 8 * nbs, nbp) ? 1 : 0;
-            b_ready = __shfl_sync(0xFFFFFFFFu, ready, 0) != 0;
+          // lookahead: the next weight stage; on the chunk's last stage the next
+          // activation stage and, on the tile's last, the next accumulator buffer
+          const uint32_t nbs = (bs + 1 == sb) ? 0u : bs + 1;
+          const uint32_t nbp = (bs + 1 == sb) ? bp ^ 1u : bp;
+          const int pr_b = probe(r.b_full + 8 * nbs, nbp);
+          int pr_a = 0, pr_acc = 0;
+          if (grp == kGrp - 1) {
+            const uint32_t nas = (as + 1 == static_cast<uint32_t>(a.SA)) ? 0u : as + 1;
+            const uint32_t nap = (as + 1 == static_cast<uint32_t>(a.SA)) ? ap ^ 1u : ap;
+            if (!kFuse || !kPair) pr_a = probe(r.a_full + 8 * nas, nap);
+            if (last && !split) {
+              const uint32_t ncs = (cs + 1 == static_cast<uint32_t>(a.acc_stages)) ? 0u : cs + 1;
+              const uint32_t ncp = (cs + 1 == static_cast<uint32_t>(a.acc_stages)) ? cp ^ 1u : cp;
+              pr_acc = probe(r.acc_empty + 8 * (ncs * kMS + kMS - 1), ncp ^ 1u);
+            }
           }
           const uint64_t b_stage = b_desc0 + bs * b_stage16;
           with_ksteps(ksteps, [&](auto KS) {
@@ -372,6 +396,11 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
           issued = true;
           commit(r.b_empty + 8 * bs);
           if (++bs == sb) { bs = 0; bp ^= 1; }
+          b_ready = seen(pr_b);
+          if (grp == kGrp - 1) {
+            a_ready = seen(pr_a);
+            acc_ready = seen(pr_acc);
+          }
         }
       }
       commit(r.a_empty + 8 * as);
