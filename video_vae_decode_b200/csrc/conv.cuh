@@ -205,10 +205,10 @@ __device__ __forceinline__ void with_ksteps(uint32_t ksteps, F&& f) {
   }
 }
 
-// MMA issuer: the whole warp 1 of the pair's leader CTA runs the loop, so
-// that the descriptor arithmetic is warp-uniform, and one elected lane issues
-// each tcgen05 instruction; lane 0 waits on the barriers and broadcasts the
-// outcome.  (Issued by a lone thread, the same MMAs measured up to twice the
+// MMA issuer: the whole warp 1 of the pair's leader CTA runs the loop; lane
+// 0 waits on the barriers and broadcasts the outcome, and one elected lane
+// issues each stage's MMAs and its commit as straight-line code.  (Issued by
+// a lone thread from run-time loops, the same MMAs measured up to twice the
 // tensor pipe's cycles each at N = 96.)  Descriptors are built once; every
 // operand start inside the rings is the base descriptor plus an offset in
 // 16-byte units (all offsets stay inside the 14-bit start-address field).  A
@@ -266,29 +266,31 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
     __syncwarp();
     return ok != 0;
   };
+  // issued by the elected lane only
   auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
-    if (elect_one()) {
-      if (kBf16) {
-        if (kPair) {
-          mma_bf16_pair(d, ad, bd, idesc, acc);
-        } else {
-          mma_bf16(d, ad, bd, idesc, acc);
-        }
-      } else if (kPair) {
-        mma_i8_pair(d, ad, bd, idesc, acc);
+    if (kBf16) {
+      if (kPair) {
+        mma_bf16_pair(d, ad, bd, idesc, acc);
       } else {
-        mma_i8(d, ad, bd, idesc, acc);
+        mma_bf16(d, ad, bd, idesc, acc);
       }
+    } else if (kPair) {
+      mma_i8_pair(d, ad, bd, idesc, acc);
+    } else {
+      mma_i8(d, ad, bd, idesc, acc);
     }
   };
-  auto commit = [&](uint32_t bar) {
-    if (elect_one()) {
-      if (kPair) {
-        mma_commit_pair_multicast(bar, 0x3);
-      } else {
-        mma_commit(bar);
-      }
+  auto commit_raw = [&](uint32_t bar) {
+    if (kPair) {
+      mma_commit_pair_multicast(bar, 0x3);
+    } else {
+      mma_commit(bar);
     }
+  };
+  // a commit issued by one elected lane of the warp
+  auto commit = [&](uint32_t bar) {
+    if (elect_one()) commit_raw(bar);
+    __syncwarp();
   };
   (void)rank;
   for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
@@ -330,22 +332,28 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
               tc_fence_after();
             }
             const uint64_t b_stage = b_desc0 + st * b_stage16;
-            with_ksteps(ksteps, [&](auto KS) {
-              constexpr int ks = decltype(KS)::value;
+            const uint32_t acc0 = acc_s;
+            if (elect_one()) {
+              with_ksteps(ksteps, [&](auto KS) {
+                constexpr int ks = decltype(KS)::value;
+                uint32_t acc_l = acc0;
 #pragma unroll
-              for (int g = 0; g < kG; ++g) {
-                const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
-                const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
-                const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4) + s * sub16;
-                const uint64_t b_tap = b_stage + g * b_tap16;
+                for (int g = 0; g < kG; ++g) {
+                  const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+                  const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+                  const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4) + s * sub16;
+                  const uint64_t b_tap = b_stage + g * b_tap16;
 #pragma unroll
-                for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
-                  mma(d_tile + s * nt, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc_s : 1u);
-                acc_s = 1u;
-              }
-            });
+                  for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
+                    mma(d_tile + s * nt, a_tap + 2 * k, b_tap + 2 * k, k == 0 ? acc_l : 1u);
+                  acc_l = 1u;
+                }
+              });
+              if (s == kMS - 1) commit_raw(r.b_empty + 8 * st);
+            }
+            __syncwarp();
+            acc_s = 1u;
             issued = true;
-            if (s == kMS - 1) commit(r.b_empty + 8 * st);
             if (++st == sb) { st = 0; sp ^= 1; }
           }
           if (last) commit(r.acc_full + 8 * s);
@@ -375,26 +383,34 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
             }
           }
           const uint64_t b_stage = b_desc0 + bs * b_stage16;
-          with_ksteps(ksteps, [&](auto KS) {
-            constexpr int ks = decltype(KS)::value;
+          // one elected lane issues the stage's MMAs as straight-line code
+          // (an election per MMA measured 18-27 % slower on the Cout = 96 layers)
+          const uint32_t acc0 = acc;
+          if (elect_one()) {
+            with_ksteps(ksteps, [&](auto KS) {
+              constexpr int ks = decltype(KS)::value;
+              uint32_t acc_l = acc0;
 #pragma unroll
-            for (int g = 0; g < kG; ++g) {
-              const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
-              const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
-              // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
-              const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
-              const uint64_t b_tap = b_stage + g * b_tap16;
+              for (int g = 0; g < kG; ++g) {
+                const uint32_t tap9 = static_cast<uint32_t>(grp * kG + g);
+                const uint32_t kh = tap9 / 3u, kw = tap9 % 3u;
+                // tap (kh, kw) of sub-tile s starts at box line (s*16 + kh)*10 + kw
+                const uint64_t a_tap = a_stage + ((kh * kGroupStride + kw * 128u) >> 4);
+                const uint64_t b_tap = b_stage + g * b_tap16;
 #pragma unroll
-              for (int s = 0; s < kMS; ++s) {
+                for (int s = 0; s < kMS; ++s) {
 #pragma unroll
-                for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
-                  mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc : 1u);
+                  for (int k = 0; k < ks; ++k)  // 32 bytes of K = 2 units
+                    mma(d_tile + s * nt, a_tap + s * sub16 + 2 * k, b_tap + 2 * k, k == 0 ? acc_l : 1u);
+                }
+                acc_l = 1u;
               }
-              acc = 1u;
-            }
-          });
+            });
+            commit_raw(r.b_empty + 8 * bs);
+          }
+          __syncwarp();
+          acc = 1u;
           issued = true;
-          commit(r.b_empty + 8 * bs);
           if (++bs == sb) { bs = 0; bp ^= 1; }
           b_ready = seen(pr_b);
           if (grp == kGrp - 1) {
@@ -934,7 +950,10 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       }
       if (++cs == static_cast<uint32_t>(a.acc_stages)) { cs = 0; cp ^= 1; }
     }
-    if (!kAcc32 && lane == 0) bulk_wait_group<0>();
+    // the last stores must have read their staging buffers before shared memory
+    // goes away; their global writes complete with the grid (a dependent launch's
+    // griddepcontrol.wait covers them)
+    if (!kAcc32 && lane == 0) bulk_wait_group_read<0>();
     if (!kAcc32 && a.out_amax) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) out_max = max(out_max, __shfl_xor_sync(0xFFFFFFFFu, out_max, o));
