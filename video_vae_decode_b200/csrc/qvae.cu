@@ -151,10 +151,16 @@ bool fit_stages_ss(Tiling* t, int want_sb) {
 // a CTA tile.  A tile is its weight stages (G taps of one 128-channel chunk
 // each), each tap MS x k-steps MMAs of 128 x NT x 32 at the measured cycles
 // per MMA for that N, plus a handshake per stage, an exposed activation load
-// per chunk when the activation ring has one stage, and the epilogue when the
-// accumulator has one buffer and its sub-tiles cannot be handed over one by
-// one.  CTA pairs load half the weights per
-// SM and measured 2-4 % faster than single CTAs of the same geometry.
+// per chunk when the activation ring has one stage, and the epilogue time an
+// accumulator buffer leaves exposed: none with two buffers (the next tile's
+// MMAs run beside it) except the last tile's; one sub-tile's with a single
+// buffer handed over sub-tile by sub-tile; all sub-tiles' otherwise.  The
+// exposed epilogue measured about 16 cycles per accumulator column and
+// sub-tile (the term that makes one sub-tile with two buffers beat two
+// sub-tiles with one on the 192-channel layers, as measured).  A CTA pair's
+// MMAs are issued once for both SMs and each SM loads half the weights: pairs
+// measured 25-40 % faster than single CTAs of the same geometry (the MMA
+// issue, not the tensor pipe, bounds the narrow layers).
 double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   double taps_t = 0;
   for (int64_t f = 0; f < std::min<int64_t>(s.T, 2); ++f) taps_t += static_cast<double>(f + 1);
@@ -162,17 +168,18 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   taps_t /= s.T;
   // cycles per MMA measured with random data: N=96 86, 128 91, 192 109, 256 143
   const double mma = std::max(0.52 * t.NT + 8.0, 60.0 + 0.17 * t.NT);
+  constexpr double kEpi = 16.0;  // exposed epilogue cycles per accumulator column and sub-tile
   const int nchunks = (s.Cin + 127) / 128;
   const double ksteps_total = s.Cin / 32.0;
   const double stages = taps_t * 9.0 / t.G * nchunks;
+  const double exposed = t.acc_stages == 2 ? 0.0 : kEpi * (t.split ? 1 : t.MS) * t.NT;
   const double per_tile = taps_t * 9.0 * ksteps_total * t.MS * mma + stages * 250.0 + 500.0 +
-                          (t.SA == 1 ? 1500.0 * taps_t * nchunks : 0.0) +
-                          (t.acc_stages == 1 && !t.split ? 6.0 * t.MS * t.NT : 0.0);
+                          (t.SA == 1 ? 1500.0 * taps_t * nchunks : 0.0) + exposed;
   const double slots = t.pair ? std::floor(sms / 2.0) : sms;
   const double waves = std::ceil(static_cast<double>(t.num_tiles) / slots);
   // the last tile's epilogue (its last sub-tile's when they are handed over one by one)
-  const double tail = t.acc_stages == 2 ? 6.0 * t.MS * t.NT : (t.split ? 6.0 * t.NT : 0.0);
-  return (waves * per_tile + tail) * (t.pair ? 0.98 : 1.0);
+  const double tail = t.acc_stages == 2 ? kEpi * t.MS * t.NT : (t.split ? kEpi * t.NT : 0.0);
+  return (waves * per_tile + tail) * (t.pair ? 1.0 : 1.3);
 }
 
 int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse) {
