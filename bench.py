@@ -666,7 +666,9 @@ def run_ours(args):
     for li, (j, p) in enumerate(zip(jobs, per_layer)):
         lops = j.s.ops()
         key = args.workload if single and len(wl.layers) == 1 else f"{args.workload}[{idx[li]}]"
-        tr = profiled_traffic(key)
+        # the committed counters describe one whole-layer launch of the two-pass
+        # kernel; the fused kernel, row bands and streamed chunks launch otherwise
+        tr = None if (j.fused or j.nb or j.chunk) else profiled_traffic(key)
         traffic.append(tr)
         numel = j.layer.x.numel()
         layer_entries.append({
