@@ -25,7 +25,7 @@
 // the halo is loaded once and reused nine times.  Temporal taps that meet a
 // causal zero frame are skipped, not computed.  Weights come pre-packed in the
 // MMA's swizzled K-major layout and stream by 2-D TMA, G taps (1, or 3 = one
-// kernel row) per pipeline stage, so the MMA thread waits and commits once per
+// kernel row) per pipeline stage, so the MMA warp waits and commits once per
 // G taps.
 //
 // CTA pairs.  With kPair the kernel runs as 2-CTA clusters on the tensor
@@ -37,8 +37,9 @@
 // of both CTAs; each CTA's epilogue drains its own TMEM rows.  No TMA load
 // uses cluster multicast.
 //
-// Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 issues
-// tcgen05.mma (one thread) and owns the TMEM allocation, warps 2-9 run the
+// Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 owns the
+// TMEM allocation and runs the MMA issue loop (the whole warp; one elected
+// lane issues each weight stage's tcgen05.mma sequence), warps 2-9 run the
 // epilogue (two per TMEM lane quarter): tcgen05.ld of their 32 TMEM lanes,
 // rescale + bias + bf16, staged through shared memory and written with TMA
 // stores.  Tiles are scheduled persistently (static stride).  With MS*NT <=
