@@ -193,6 +193,20 @@ def test_conv_few_ctas_many_tiles_exact(q, tiling):
         q.qvae_set_conv_cta_limit(0)
 
 
+@pytest.mark.parametrize("Cin", [32, 96, 160, 192])
+@pytest.mark.parametrize("tiling", [dict(mode=2, MS=2, NT=96, G=3), dict(mode=1, MS=1, NT=96, G=3, SB=2)])
+def test_conv_one_pair_every_kstep_count_exact(q, Cin, tiling):
+    # one CTA pair (or two single CTAs) walks every tile, so the MMA warp's
+    # lookahead probes of the next weight stage, activation stage and
+    # accumulator buffer cross chunk, tile and ring boundaries many times;
+    # the last 128-channel chunk has 1, 3, 1 and 2 k-steps of 32 channels
+    q.qvae_set_conv_cta_limit(2)
+    try:
+        assert conv_case(q, synth.LayerShape(Cin, 96, 21, 19, T=3), seed=Cin, tiling=tiling) == 1.0
+    finally:
+        q.qvae_set_conv_cta_limit(0)
+
+
 @pytest.mark.parametrize("tiling", TILINGS)
 def test_conv_tilings_exact(q, tiling):
     # spans several tiles in h, w and channels, with ragged edges and T > 2
