@@ -51,7 +51,8 @@ typedef enum qvae_status {
   QVAE_ERR_ALIGN = 3,    /* a pointer is not 16-byte aligned */
   QVAE_ERR_CUDA = 4,     /* a CUDA call or kernel launch failed */
   QVAE_ERR_TIMEOUT = 5,  /* a device-side pipeline wait ran out of time */
-  QVAE_ERR_UNSUPPORTED = 6
+  QVAE_ERR_UNSUPPORTED = 6,
+  QVAE_ERR_BOUNDS = 7    /* (debug builds only) a load or store failed its bounds check and was skipped */
 } qvae_status;
 
 /* Shape of one CausalConv3d layer; input and output have the same N, T, H, W. */
@@ -353,7 +354,10 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
 /*
  * Waits for `stream`, then returns and clears the device error word:
  * QVAE_OK, QVAE_ERR_TIMEOUT (a pipeline wait inside a kernel gave up; the
- * results of that call are invalid), or QVAE_ERR_CUDA if the wait failed.
+ * results of that call are invalid), QVAE_ERR_BOUNDS (a library built with
+ * -DQVAE_DEBUG_CHECKS found a load or store outside its tensor, ring or
+ * accumulator and skipped it; the results are invalid), or QVAE_ERR_CUDA if
+ * the wait failed.
  */
 int qvae_get_error(void* stream);
 
@@ -370,6 +374,13 @@ int qvae_set_wait_limit_ns(uint64_t limit_ns);
  * QVAE_ERR_TIMEOUT.  Exercises the timeout path without faulting the GPU.
  */
 int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
+ * How this library was built: bit 0 set = the kernels' bounds checks are
+ * compiled in (libqvae_debug.so, -DQVAE_DEBUG_CHECKS; a failed check makes
+ * qvae_get_error() return QVAE_ERR_BOUNDS).  Other bits are zero.
+ */
+int qvae_build_flags(void);
 
 /*
  * Convolution tiling override for tuning and tests (process-wide, not

@@ -31,10 +31,16 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_release_library_has_no_debug_checks():
+    # the in-tree library is the release build unless QVAE_LIBRARY names another
+    if not os.environ.get("QVAE_LIBRARY"):
+        assert qvae.lib().qvae_build_flags() == 0
+
+
 def test_status_strings():
     L = qvae.lib()
-    for code in range(7):
-        assert L.qvae_status_string(code)
+    for code in range(8):
+        assert L.qvae_status_string(code) not in (None, b"", b"unknown status")
     assert L.qvae_status_string(99) == b"unknown status"
 
 

@@ -298,6 +298,11 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
     const int nkb = tile_nkb(tile);
     const uint32_t d_tile = r.tmem_base + cs * static_cast<uint32_t>(kMS) * nt;
     const uint32_t accb = cs * static_cast<uint32_t>(kMS);  // this buffer's first barrier index
+    if (!check_bounds((cs + 1u) * static_cast<uint32_t>(kMS) * nt <= a.tmem_cols &&
+                      accb + static_cast<uint32_t>(kMS) <= static_cast<uint32_t>(kAccBars))) {
+      *abort_flag = 1;
+      return false;
+    }
     if (!split) {
       // the epilogue warps release a buffer's sub-tiles in order: the last one's
       // barrier completing implies the others'
@@ -540,6 +545,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         const int tap = kt * 9 + grp * a.G + g;  // (kt * 3 + kh) * 3 + kw
         const int row = (tap * a.nchunks + ch) * a.Cout + c.co0 + static_cast<int>(rank) * (a.NT / 2);
         const uint32_t dst = b_ring + bs * a.b_stage_bytes + static_cast<uint32_t>(g) * a.b_tap_bytes;
+        const int rows = kPair ? a.NT / 2 : a.NT;
+        if (!check_bounds(tap >= 0 && tap < 27 && ch >= 0 && ch < a.nchunks && row >= 0 &&
+                          row + rows <= 27 * a.nchunks * a.Cout &&
+                          dst + a.b_tap_bytes <= b_ring + static_cast<uint32_t>(a.SB) * a.b_stage_bytes))
+          continue;
         if (kPair) {
           tma_load_2d_pair(dst, &tmap_w, map_to_cta(bar, 0), 0, row);
         } else {
@@ -569,7 +579,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
           if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
           const uint32_t bar = a_full + 8 * as;
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
-          if (kPair) {
+          // the channel coordinate (the box's innermost) must sit on a 16-byte boundary
+          if (!check_bounds(ch >= 0 && ch < a.nchunks && (ch * 128) % 16 == 0 && frame >= 0 &&
+                            frame < a.T + 2 * a.carry && c.n >= 0 && c.n < a.N && c.w0 >= 0 && c.w0 < a.W &&
+                            c.h0 >= 0 && a.a_box_bytes <= a.a_stage_bytes && as < static_cast<uint32_t>(a.SA))) {
+          } else if (kPair) {
             tma_load_5d_pair(a_ring + as * a.a_stage_bytes, &tmap_x, map_to_cta(bar, 0), ch * a.chunk_elems,
                              c.w0 - 1, c.h0 - 1 + a.halo_top, frame, c.n);
           } else {
@@ -681,6 +695,10 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       const int frame = p.c.t + kt - 2 + 2 * a.carry;
       const uint32_t bar = stg_full + 8 * slot;
       mbar_arrive_expect_tx(bar, a.stg_slot_bytes);
+      if (!check_bounds(ch >= 0 && ch < a.nchunks && frame >= 0 && frame < a.T + 2 * a.carry && p.c.n >= 0 &&
+                        p.c.n < a.N && p.c.w0 >= 0 && p.c.w0 < a.W && slot < static_cast<uint32_t>(a.SS) &&
+                        (p.g + 1) * a.stg_rows <= 16 * a.MS + 2))
+        return;
       tma_load_5d(stg_ring + slot * a.stg_slot_bytes, &tmap_x, bar, ch * 128, p.c.w0 - 1,
                   p.c.h0 - 1 + a.halo_top + p.g * a.stg_rows, frame, p.c.n);
     };
@@ -850,13 +868,17 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         }
         tc_fence_after();
         const uint32_t t_sub = t_buf + static_cast<uint32_t>(s * a.NT);
+        if (!check_bounds((accb + static_cast<uint32_t>(s) + 1u) * static_cast<uint32_t>(a.NT) <= a.tmem_cols)) {
+          dead = true;
+          break;
+        }
         auto issue = [&](int jj, uint32_t(&v)[32]) { tmem_ld_32x32b_x32(t_sub + static_cast<uint32_t>(jj << 5), v); };
         auto process = [&](int jj, const uint32_t(&v)[32]) {
           const int cc = jj << 5;
           if (kAcc32) {
             const int h = c.h0 + s * kTileRows + row / kTileW;
             const int w = c.w0 + row % kTileW;
-            if (h < a.H && w < a.W) {
+            if (h < a.H && w < a.W && check_bounds(c.co0 + cc + 32 <= a.Cout && c.n < a.N && c.t < a.T)) {
               const int64_t pix = ((static_cast<int64_t>(c.n) * a.T + c.t) * a.H + h) * a.W + w;
               int4* dst = reinterpret_cast<int4*>(a.acc_out + pix * a.Cout + c.co0 + cc);
 #pragma unroll
@@ -917,7 +939,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_5d(&tmap_out, sbuf, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
+              // a box that starts below the last row is clipped whole by the tensor map
+              if (check_bounds((c.co0 + cc) % 8 == 0 && c.co0 + cc + 32 <= a.Cout && c.w0 >= 0 && c.w0 < a.W &&
+                               c.h0 + s * kTileRows + q * 4 >= 0 && c.t < a.T && c.n < a.N &&
+                               sbuf + kEpiBufBytes <= epi_stage + static_cast<uint32_t>(kEpiWarps * a.epi_bufs) * kEpiBufBytes))
+                tma_store_5d(&tmap_out, sbuf, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
               bulk_commit_group();
             }
             if (a.epi_bufs == 2) buf ^= 1u;

@@ -97,7 +97,25 @@ enum DeviceError : int {
   kErrTimeoutEpilogue = 0x103,
   kErrTimeoutDrain = 0x104,
   kErrTimeoutConvert = 0x105,
+  kErrBounds = 0x106,  // a debug build found a load or store outside its tensor or ring
 };
+
+// Debug builds (-DQVAE_DEBUG_CHECKS) check each TMA load's and store's
+// coordinates and shared-memory range, each direct store's index and each
+// MMA's accumulator columns before issuing them.  A failed check records
+// kErrBounds in the error word and the access is skipped -- no trap: the
+// bounded waits then let the kernel finish (a skipped load leaves its
+// barrier short, so the waits give up and the kernel drains and returns).
+// Release builds compile the checks away.
+__device__ __forceinline__ bool check_bounds(bool ok) {
+#ifdef QVAE_DEBUG_CHECKS
+  if (!ok) atomicCAS(&g_qvae_error, 0, static_cast<int>(kErrBounds));
+  return ok;
+#else
+  (void)ok;
+  return true;
+#endif
+}
 
 // Wait for the phase with the given parity to complete.  Returns false when
 // the CTA has been told to abort or when this wait ran past `limit_ns`.

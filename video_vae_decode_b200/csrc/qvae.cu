@@ -615,6 +615,7 @@ const char* qvae_status_string(int status) {
     case QVAE_ERR_CUDA: return "CUDA error";
     case QVAE_ERR_TIMEOUT: return "device-side wait timed out";
     case QVAE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QVAE_ERR_BOUNDS: return "a device bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -936,6 +937,11 @@ int qvae_get_error(void* stream) {
     const int zero = 0;
     QVAE_CUDA(cudaMemcpyToSymbol(qvae::g_qvae_error, &zero, sizeof zero));
     char buf[64];
+    if (v == qvae::kErrBounds) {
+      std::snprintf(buf, sizeof buf, "device bounds check failed (code 0x%x)", v);
+      t_last_error = buf;
+      return QVAE_ERR_BOUNDS;
+    }
     std::snprintf(buf, sizeof buf, "device wait timed out (code 0x%x)", v);
     t_last_error = buf;
     return QVAE_ERR_TIMEOUT;
@@ -947,6 +953,14 @@ int qvae_set_wait_limit_ns(uint64_t limit_ns) {
   if (limit_ns == 0) return QVAE_ERR_ARG;
   g_wait_limit_ns = limit_ns;
   return QVAE_OK;
+}
+
+int qvae_build_flags(void) {
+#ifdef QVAE_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 int qvae_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

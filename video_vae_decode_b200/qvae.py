@@ -15,10 +15,12 @@ from typing import Optional, Sequence
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libqvae.so")
+# QVAE_LIBRARY names another build of the same ABI (libqvae_debug.so: the
+# bounds-checked kernels); the default is the in-tree release library.
+LIB_PATH = os.environ.get("QVAE_LIBRARY") or os.path.join(HERE, "libqvae.so")
 
 QVAE_OK, QVAE_ERR_ARG, QVAE_ERR_SHAPE, QVAE_ERR_ALIGN = 0, 1, 2, 3
-QVAE_ERR_CUDA, QVAE_ERR_TIMEOUT, QVAE_ERR_UNSUPPORTED = 4, 5, 6
+QVAE_ERR_CUDA, QVAE_ERR_TIMEOUT, QVAE_ERR_UNSUPPORTED, QVAE_ERR_BOUNDS = 4, 5, 6, 7
 
 # Every symbol include/qvae.h declares.
 EXPORTS = (
@@ -26,7 +28,7 @@ EXPORTS = (
     "qvae_quantize_weights", "qvae_act_workspace_bytes", "qvae_act_absmax_quant",
     "qvae_causal_conv3d_w8a8", "qvae_causal_conv3d_w8a8_acc32", "qvae_decode_workspace_bytes",
     "qvae_decode_layers", "qvae_get_error", "qvae_set_wait_limit_ns",
-    "qvae_selftest_wait_timeout", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
+    "qvae_selftest_wait_timeout", "qvae_build_flags", "qvae_set_conv_tiling", "qvae_get_conv_tiling", "qvae_set_conv_cta_limit",
     "qvae_act_absmax_quant_noalloc",
     "qvae_causal_conv3d_w8a8_carry", "qvae_causal_conv3d_w8a8_carry_acc32",
     "qvae_act_absmax", "qvae_act_quant_from_absmax",
@@ -95,6 +97,7 @@ def lib():
             "qvae_get_error": ([p], ctypes.c_int),
             "qvae_set_wait_limit_ns": ([u64], ctypes.c_int),
             "qvae_selftest_wait_timeout": ([u64, p], ctypes.c_int),
+            "qvae_build_flags": ([], ctypes.c_int),
             "qvae_set_conv_tiling": ([i32, i32, i32, i32, i32, i32], ctypes.c_int),
             "qvae_set_conv_cta_limit": ([i32], ctypes.c_int),
             "qvae_set_fused_quant": ([i32], ctypes.c_int),
