@@ -70,6 +70,8 @@ def parse():
                          "absmax, then per band quantise + band convolution)")
     ap.add_argument("--split", action="store_true",
                     help="split one image layer across the ranks by row bands (strong scaling)")
+    ap.add_argument("--native", action="store_true",
+                    help="time the native-precision (bf16 kind::f16) convolution of the workload's layers")
     ap.add_argument("--fused", action="store_true",
                     help="layers as absmax + the convolution quantising its bf16 input in the kernel")
     ap.add_argument("--chain", default="",
@@ -797,6 +799,107 @@ def run_split(args):
     return 0
 
 
+def run_native(args):
+    """The native-precision convolution (bf16 operands on kind::f16, fp32
+    accumulators, bf16 output: the layers the release note keeps unquantised)
+    over the workload's layers on one GPU, in TFLOP/s against the bf16 peak.
+
+    A step is every layer's convolution (no activation passes: the layer reads
+    bf16 x directly).  Buffer sets larger than 3x L2 rotate; one CUDA graph per
+    set; per-layer CUDA-event times from a second pass behind a GPU spin.
+    """
+    import math
+    import statistics
+    import torch
+    from video_vae_decode_b200 import qvae, synth
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--native runs on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    qvae.lib()
+    wl = synth.WORKLOADS[args.workload]
+    idx = [args.layer] if args.layer >= 0 else list(range(len(wl.layers)))
+    layers = synth.draw_workload(args.workload, only=idx)
+    layers = [layers[i] for i in idx] if len(layers) > len(idx) else layers
+    packed = [qvae.pack_weights_bf16(l.w.to(dev)) for l in layers]
+    bias = [l.bias.to(dev) for l in layers]
+    per_set = sum(l.x.numel() * 2 + l.shape.pixels * l.shape.Cout * 2 for l in layers)
+    n_sets = max(2, math.ceil(3 * 126e6 / per_set))
+    sets = [[dict(x=l.x.to(dev), out=torch.empty((l.shape.N, l.shape.T, l.shape.H, l.shape.W, l.shape.Cout),
+                                                dtype=torch.bfloat16, device=dev)) for l in layers]
+            for _ in range(n_sets)]
+    stream = torch.cuda.Stream(device=dev)   # graphs are captured on a side stream
+
+    def step(ss):
+        for st, wp, b in zip(ss, packed, bias):
+            qvae.qvae_causal_conv3d_bf16(st["x"], wp, b, st["out"], stream)
+
+    with torch.cuda.stream(stream):
+        step(sets[0])
+    torch.cuda.synchronize()
+    graphs = []
+    for ss in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(ss)
+        graphs.append(g)
+    with torch.cuda.stream(stream):            # replays launch on the current stream
+        for i in range(max(args.warmup, 3)):
+            graphs[i % n_sets].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk, torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % n_sets].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if qvae.qvae_get_error() != 0:
+        raise RuntimeError("device-side timeout")
+    ms = e0.elapsed_time(e1) / args.steps
+    R = max(10, min(args.steps, 100))
+    per_layer = []
+    for li, l in enumerate(layers):
+        ts = []
+        with torch.cuda.stream(stream):
+            for i in range(R):
+                st = sets[i % n_sets][li]
+                torch.cuda._sleep(SPIN_CYCLES)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                qvae.qvae_causal_conv3d_bf16(st["x"], packed[li], bias[li], st["out"], stream)
+                b.record(stream)
+                ts.append((a, b))
+        torch.cuda.synchronize()
+        t = statistics.mean(a.elapsed_time(b) for a, b in ts)
+        per_layer.append({"layer": layer_name(l), "ms": t, "tflops": l.shape.ops() / (t * 1e-3) / 1e12,
+                          "tiling": qvae.qvae_get_conv_tiling(l.shape.N, l.shape.T, l.shape.H, l.shape.W,
+                                                              l.shape.Cin, l.shape.Cout, 2)})
+    ops = sum(l.shape.ops() for l in layers)
+    bf16_burst, _, peak_src = measured_peaks()
+    conv_sum = sum(p["ms"] for p in per_layer)
+    achieved = ops / (conv_sum * 1e-3) / 1e12
+    line = {
+        "metric": "native-precision CausalConv3d TFLOP/s (bf16 operands, fp32 accumulation, bf16 out)",
+        "value": ops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": args.workload, "layers": [layer_name(l) for l in layers],
+                   "arithmetic": "bf16 x bf16 products, fp32 accumulation, fp32 bias add, bf16 out",
+                   "l2": f"inputs and outputs rotate over {n_sets} buffer sets (> 3x the 126 MB L2)",
+                   "launch": "one CUDA graph replay per step (one convolution per layer)"},
+        "per_layer": per_layer,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16_burst, "unit": "TFLOP/s",
+                     "frac": achieved / bf16_burst, "traffic": None, "peak_source": peak_src,
+                     "kernel": "conv3d_bf16_kernel"},
+        "gpu_launches": args.steps * len(layers),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def run_chain(args):
     """Layers of a workload as one qvae_decode_layers chain on one GPU.
 
@@ -894,6 +997,8 @@ def main():
         return run_chain(args)
     if args.split:
         return run_split(args)
+    if args.native:
+        return run_native(args)
     return run_ours(args)
 
 
