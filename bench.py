@@ -702,7 +702,7 @@ def run_ours(args):
             "conv_frac": lops / (p["conv"] * 1e-3) / 1e12 / peak,
             "act_gbs": (2 if (j.fused or j.overlap) else 5) * numel / (p["act"] * 1e-3) / 1e9,
             "tiling": qvae.qvae_get_conv_tiling(j.s.N, j.s.T, j.s.H, j.s.W, j.s.Cin, j.s.Cout,
-                                                1 if j.fused else (3 if j.overlap else 0)),
+                                                1 if j.fused else 0),
             "dram_bytes_per_conv_launch": tr})
     traffic_mean = (sum(traffic) / len(traffic)) if all(t is not None for t in traffic) else None
     h2d = sum(j.layer.x.numel() * 2 for j in jobs)

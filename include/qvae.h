@@ -456,7 +456,7 @@ int qvae_set_fused_quant(int32_t on);
  * NT, SA, SB, accumulator buffers (1 or 2), CTAs of work, mode (1 or 2), G.
  * variant: 0 the W8A8 convolution of INT8 codes, 1 the fused W8A8
  * convolution (bf16 input quantised in the kernel), 2 the native-precision
- * convolution, 3 the convolution of qvae_layer_w8a8 (overlapped quantisation). */
+ * convolution. */
 int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8);
 
 #if defined(__GNUC__)

@@ -5,9 +5,8 @@ Codes, scale, INT32 accumulators and bf16 outputs must all be bit-identical
 to the oracle's -- the same bar as the two-call path (qvae_act_absmax_quant +
 qvae_causal_conv3d_w8a8), whose codes and scale this path reproduces.  The
 cases cover several tiles and ragged edges, CTA pairs and single CTAs, few
-CTAs walking many tiles (the band waits and unit claims interleave), bands
-across frames and batch items, more input rows than 16 x the band counters,
-T > 2 and N > 1, the
+CTAs walking many tiles (the band waits and unit claims interleave), more
+input rows than band counters (several rows per band), T > 2 and N > 1, the
 full-size decoder layers, and the argument errors.
 """
 import numpy as np
@@ -89,7 +88,7 @@ def test_layer_overlap_tiny_and_odd(q, H, W, T):
 
 
 @pytest.mark.parametrize("tiling,ctas", [(dict(mode=1, MS=1), 3), (dict(mode=2, MS=1, G=3), 2),
-                                         (dict(mode=2, MS=2, NT=96, G=3), 4), (dict(mode=1, MS=4, NT=32), 1)])
+                                         (dict(mode=2, MS=2, NT=96, G=3), 4), (dict(mode=1, MS=4, NT=64), 1)])
 def test_layer_overlap_few_ctas_many_tiles(q, tiling, ctas):
     # few CTAs: each producer walks many tiles and band waits, and the few
     # quantising warps claim every unit of the tensor
@@ -97,15 +96,9 @@ def test_layer_overlap_few_ctas_many_tiles(q, tiling, ctas):
                          tiling=tiling, ctas=ctas)
 
 
-def test_layer_overlap_bands_across_frames_and_items(q):
-    # 2 x 3 x 700 = 4200 input rows in bands of 16: bands cross frame and
-    # batch-item boundaries, and the last band is short
+def test_layer_overlap_several_rows_per_band(q):
+    # 2 x 3 x 700 = 4200 input rows > 4095 band counters: two rows per band
     check_against_oracle(q, synth.draw_custom(synth.LayerShape(32, 32, 700, 9, T=3, N=2), seed=4))
-
-
-def test_layer_overlap_more_rows_than_band_counters(q):
-    # 16 x 4100 = 65600 input rows > 16 x 4095: 17 rows per band
-    check_against_oracle(q, synth.draw_custom(synth.LayerShape(32, 32, 4100, 1, T=1, N=16), seed=6))
 
 
 def test_layer_overlap_outliers_and_zero(q):

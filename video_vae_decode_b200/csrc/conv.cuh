@@ -138,18 +138,11 @@ constexpr int kMaxStgSlots = 8;
 constexpr uint32_t kStgPixelBytes = 256;            // 128 bf16 channels of one pixel
 constexpr uint32_t kEpiBufBytes = 2048;    // one epilogue staging buffer: 32 pixels x 64 B
 constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
-// Overlapped quantisation: a unit is 128 groups of 16 values (4 KB of bf16 in,
-// 2 KB of codes out), moved by bulk copies through a per-warp shared-memory
-// ring of kOvlInSlots input and kOvlOutSlots output slots; a warp claims
-// kClaimUnits units at a time.
-constexpr int kUnitGroups = 128;
-constexpr uint32_t kClaimUnits = 8;
-constexpr int kOvlInSlots = 3;
-constexpr int kOvlOutSlots = 2;
-constexpr uint32_t kOvlInBytes = kUnitGroups * 32;   // bf16
-constexpr uint32_t kOvlOutBytes = kUnitGroups * 16;  // codes
-constexpr uint32_t kOvlWarpBytes = kOvlInSlots * kOvlInBytes + kOvlOutSlots * kOvlOutBytes;
-constexpr uint32_t kOvlBytes = kCvtWarps * kOvlWarpBytes;  // a multiple of 1024
+// Streamed quantisation: a unit is 8 groups of 16 values per lane of a warp
+// (8 KB of bf16 in, 4 KB of codes out); a warp claims kClaimUnits units at a time.
+constexpr int kUnitLaneGroups = 8;
+constexpr int kUnitGroups = 32 * kUnitLaneGroups;
+constexpr uint32_t kClaimUnits = 4;
 
 // Packed fp32 pairs (low word = first value).  RN(a * b); and RN(a + b)
 // computed as fma(a, one, b) with `one` = (1.0, 1.0) from a kernel argument:
@@ -496,8 +489,8 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
 
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
-  const uint32_t stg_ring = b_ring + a.SB * a.b_stage_bytes;  // fused: bf16 row groups; overlapped: unit rings
-  const uint32_t epi_stage = stg_ring + (kFuse ? a.SS * a.stg_slot_bytes : kOverlap ? kOvlBytes : 0u);  // 1024-aligned
+  const uint32_t stg_ring = b_ring + a.SB * a.b_stage_bytes;                     // fused: bf16 row groups
+  const uint32_t epi_stage = stg_ring + (kFuse ? a.SS * a.stg_slot_bytes : 0u);  // 1024-aligned
   const uint32_t bars = epi_stage + kEpiWarps * a.epi_bufs * kEpiBufBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
@@ -534,9 +527,6 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         mbar_init(stg_full + 8 * i, 1);
         asm volatile("st.shared.u32 [%0], 0;" ::"r"(stg_done + 8 * i) : "memory");
       }
-    }
-    if (kOverlap) {
-      for (int i = 0; i < kCvtWarps * kOvlInSlots; ++i) mbar_init(stg_full + 8 * i, 1);  // input slots
     }
     for (int i = 0; i < a.SB; ++i) {
       mbar_init(b_full + 8 * i, 1);
@@ -708,18 +698,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     __syncwarp();
   } else if (kOverlap && warp >= 2 + kEpiWarps) {
     // ------------------------------------------------ overlapped quantisers
-    // Each of the two warps runs its own ring: lane 0 claims units, loads a
-    // unit's bf16 into an input slot with one bulk copy (kOvlInSlots units in
-    // flight), the whole warp converts it into an output slot, and lane 0
-    // stores the codes with one bulk copy.  A unit's band is released once
-    // its store has completed (bulk-group wait, then a release add), one unit
-    // behind, so no lane ever waits on a global store or load.  Claims go out
-    // in unit order, so every band below the claim frontier belongs to a
-    // warp that is running.
-    const int cw = warp - (2 + kEpiWarps);
-    const uint32_t in_ring = stg_ring + static_cast<uint32_t>(cw) * kOvlWarpBytes;
-    const uint32_t out_ring = in_ring + kOvlInSlots * kOvlInBytes;
-    const uint32_t in_full = stg_full + 8u * static_cast<uint32_t>(cw * kOvlInSlots);
+    // Unit u: band u / band_units, groups [g0, g1) of it (at most 256); lane
+    // l takes groups g0 + l + 32k.  The loads of a unit are issued before the
+    // previous unit is released, so the release's wait for the earlier stores
+    // overlaps them.  Claims go out in unit order, so every band below the
+    // claim frontier belongs to a warp that is running.
     grid_dependency_wait();  // the partial maxima and the zeroed counters are final
     uint32_t m = 0;
     for (int k = lane; k < a.npartial; k += 32) m = max(m, __ldcg(a.partial + k));
@@ -728,8 +711,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     const float sa = __fdiv_rn(bf16_bits_to_f32(m) * 1.0f, 127.0f);  // clip ratio 1.0
     const Quantizer z = make_quantizer(sa);
     const bool zero_scale = sa == 0.0f;
-    if (blockIdx.x == 0 && cw == 0 && lane == 0 && a.x_scale_out) *a.x_scale_out = sa;
-    constexpr uint32_t kEnd = 0xFFFFFFFFu;
+    if (blockIdx.x == 0 && warp == 2 + kEpiWarps && lane == 0 && a.x_scale_out) *a.x_scale_out = sa;
     const uint32_t nclaims = (a.total_units + kClaimUnits - 1) / kClaimUnits;
     const uint32_t claim_stride = gridDim.x * static_cast<uint32_t>(kCvtWarps);
     auto unit_range = [&](uint32_t unit, int64_t& g0, int64_t& g1) -> int {
@@ -738,23 +720,23 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       g1 = min(min(g0 + kUnitGroups, (b + 1) * a.band_groups), a.total_groups);
       return b;
     };
-    // lane 0's claim state; the next claim is taken one claim early, so the
-    // atomic's latency is hidden behind the current claim's units
-    uint32_t claim_u = 0, claim_end = 0, claim_next = 0;
-    bool claims_done = false;
-    if (lane == 0) claim_next = atomicAdd(a.next_claim, 1u);
-    auto next_unit = [&]() -> uint32_t {
-      if (claims_done) return kEnd;
-      if (claim_u == claim_end) {
-        const uint32_t c = claim_next;
-        if (c >= nclaims) {
-          claims_done = true;
-          return kEnd;
-        }
-        claim_next = atomicAdd(a.next_claim, 1u);
-        claim_u = c * kClaimUnits;
-        claim_end = min(claim_u + kClaimUnits, a.total_units);
-        if (c + claim_stride < nclaims) {
+    auto release = [&](int b) {
+      __syncwarp();  // every lane's stores are ordered before lane 0's release
+      if (lane == 0 && check_bounds(b >= 0 && static_cast<int64_t>(b) * a.band_units < a.total_units))
+        red_release_gpu_add(a.band_done + b, 1u);
+      __syncwarp();
+    };
+    int pend = -1;
+    uint32_t u = 0, u_end = 0;
+    while (true) {
+      if (u == u_end) {
+        uint32_t c = 0;
+        if (lane == 0) c = atomicAdd(a.next_claim, 1u);
+        c = __shfl_sync(0xFFFFFFFFu, c, 0);
+        if (c >= nclaims) break;
+        u = c * kClaimUnits;
+        u_end = min(u + kClaimUnits, a.total_units);
+        if (lane == 0 && c + claim_stride < nclaims) {
           // bring the claim about one round ahead into L2 for the warp that will take it
           const uint32_t p0 = (c + claim_stride) * kClaimUnits;
           const uint32_t p1 = min(p0 + kClaimUnits, a.total_units) - 1;
@@ -764,114 +746,27 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
           if (l1 > f0) prefetch_l2(a.x_in + 2 * f0, static_cast<uint32_t>((l1 - f0) * 32));
         }
       }
-      return claim_u++;
-    };
-    // lane 0: a unit into input slot `slot` (an end marker or an empty unit completes the phase without bytes)
-    auto load_unit = [&](uint32_t slot, uint32_t unit) {
-      const uint32_t bar = in_full + 8u * slot;
-      int64_t g0 = 0, g1 = 0;
-      if (unit != kEnd) unit_range(unit, g0, g1);
-      if (g1 <= g0) {
-        mbar_arrive(bar);
-        return;
-      }
-      const uint32_t bytes = static_cast<uint32_t>(g1 - g0) * 32u;
-      mbar_arrive_expect_tx(bar, bytes);
-      if (check_bounds(g0 >= 0 && g1 <= a.total_groups && bytes <= kOvlInBytes && slot < kOvlInSlots))
-        bulk_load(in_ring + slot * kOvlInBytes, a.x_in + 2 * g0, bytes, bar);
-    };
-    // units in the input slots, oldest first (lane 0)
-    uint32_t q0 = kEnd, q1 = kEnd, q2 = kEnd;
-    static_assert(kOvlInSlots == 3, "the unit queue below holds three slots");
-    if (lane == 0) {
-      q0 = next_unit();
-      load_unit(0, q0);
-      q1 = next_unit();
-      load_unit(1, q1);
-      q2 = next_unit();
-      load_unit(2, q2);
-    }
-    // bands of the units whose stores are the newest kRelLag in flight, newest first (lane 0)
-    constexpr int kRelLag = 6;
-    int pend[kRelLag];
-#pragma unroll
-    for (int i = 0; i < kRelLag; ++i) pend[i] = -1;
-    // input slots whose load may still be in flight, and the parity of that load's phase (lane 0)
-    uint32_t armed = (q0 != kEnd ? 1u : 0u) | (q1 != kEnd ? 2u : 0u) | (q2 != kEnd ? 4u : 0u), apar = 0;
-    auto release = [&](int b) {
-      fence_proxy_async_global();  // the codes were written by the async proxy
-      if (check_bounds(b >= 0 && static_cast<int64_t>(b) * a.band_units < a.total_units))
-        red_release_gpu_add(a.band_done + b, 1u);
-    };
-    for (uint32_t k = 0;; ++k) {
-      const uint32_t unit = __shfl_sync(0xFFFFFFFFu, q0, 0);
-      if (unit == kEnd) break;
-      const uint32_t slot = k % kOvlInSlots, par = (k / kOvlInSlots) & 1u, oslot = k % kOvlOutSlots;
-      int ok = 1;
-      if (lane == 0) {
-        ok = mbar_wait(in_full + 8u * slot, par, abort_flag, limit, kErrTimeoutConvert);
-        if (ok) armed &= ~(1u << slot);
-        bulk_wait_group_read<kOvlOutSlots - 1>();  // the store that last used this output slot has read it
-      }
-      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
-      __syncwarp();
       int64_t g0, g1;
-      const int b = unit_range(unit, g0, g1);
-      const int n = static_cast<int>(g1 - g0);
-      const uint32_t src = in_ring + slot * kOvlInBytes, dst = out_ring + oslot * kOvlOutBytes;
-      for (int j = lane; j < n; j += 32) {
-        uint4 va, vb;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(va.x), "=r"(va.y), "=r"(va.z), "=r"(va.w)
-                     : "r"(src + static_cast<uint32_t>(j) * 32u));
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(vb.x), "=r"(vb.y), "=r"(vb.z), "=r"(vb.w)
-                     : "r"(src + static_cast<uint32_t>(j) * 32u + 16u));
-        const uint4 c = quant16_x2(z, zero_scale, va, vb);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + static_cast<uint32_t>(j) * 16u),
-                     "r"(c.x), "r"(c.y), "r"(c.z), "r"(c.w)
-                     : "memory");
-      }
-      fence_proxy_async_smem();  // the codes are read by the bulk store (async proxy)
-      __syncwarp();
-      if (lane == 0) {
-        if (n > 0 && check_bounds(g0 >= 0 && g1 <= a.total_groups))
-          bulk_store(a.xq_out + g0, dst, static_cast<uint32_t>(n) * 16u);
-        bulk_commit_group();
-        // the input slot is free: load the unit three ahead
-        const uint32_t nu = next_unit();
-        load_unit(slot, nu);
-        if (nu != kEnd) {
-          armed |= 1u << slot;
-          apar = (apar & ~(1u << slot)) | ((par ^ 1u) << slot);  // the slot's next use is k + 3
+      const int b = unit_range(u, g0, g1);
+      ++u;
+      uint4 va[kUnitLaneGroups], vb[kUnitLaneGroups];
+#pragma unroll
+      for (int k = 0; k < kUnitLaneGroups; ++k) {
+        const int64_t g = g0 + lane + 32 * k;
+        if (g < g1) {
+          va[k] = __ldcs(a.x_in + 2 * g);
+          vb[k] = __ldcs(a.x_in + 2 * g + 1);
         }
-        q0 = q1;
-        q1 = q2;
-        q2 = nu;
-        // every store but the newest kRelLag has completed: release the band of
-        // the unit kRelLag back (output slots are reused once read, much earlier)
-        bulk_wait_group<kRelLag>();
-        if (pend[kRelLag - 1] >= 0) release(pend[kRelLag - 1]);
-#pragma unroll
-        for (int i = kRelLag - 1; i > 0; --i) pend[i] = pend[i - 1];
-        pend[0] = b;
       }
-      __syncwarp();
-    }
-    if (lane == 0) {
-      bulk_wait_group<0>();
-      if (!*abort_flag) {
+      if (pend >= 0) release(pend);
 #pragma unroll
-        for (int i = 0; i < kRelLag; ++i)
-          if (pend[i] >= 0) release(pend[i]);
-      } else {
-        // let the input loads still in flight land before the CTA exits
-        int dummy = 0;
-        for (uint32_t i = 0; i < kOvlInSlots; ++i)
-          if (armed >> i & 1u) mbar_wait(in_full + 8u * i, apar >> i & 1u, &dummy, limit, kErrTimeoutDrain);
+      for (int k = 0; k < kUnitLaneGroups; ++k) {
+        const int64_t g = g0 + lane + 32 * k;
+        if (g < g1 && check_bounds(g >= 0 && g < a.total_groups)) a.xq_out[g] = quant16_x2(z, zero_scale, va[k], vb[k]);
       }
+      pend = b;
     }
-    __syncwarp();
+    if (pend >= 0) release(pend);
   } else if (kFuse && warp >= 2 + kEpiWarps) {
     // ----------------------------------------------------------- quantisers
     // The activation boxes of the fused variant, in the MMA's order: each

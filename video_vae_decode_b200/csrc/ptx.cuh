@@ -217,14 +217,6 @@ __device__ __forceinline__ void tma_store_5d(const void* tmap, uint32_t src, int
       : "memory");
 }
 
-// Contiguous shared -> global copy, completing with the thread's bulk groups
-// (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
-               "r"(src), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

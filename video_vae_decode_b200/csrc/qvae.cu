@@ -89,7 +89,6 @@ struct Tiling {
   bool split;    // per-sub-tile accumulator hand-off
   int epi_bufs;  // epilogue staging buffers per warp
   bool fuse;     // quantisation in the kernel: a bf16 staging ring of SS row groups
-  bool overlap;  // the overlapped variant: two quantising warps' unit rings
   int SS;
   uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
   int tiles_w, tiles_h, tiles_n, num_tiles, ctas_per_tile;
@@ -104,7 +103,6 @@ constexpr uint32_t kStgSlotBytes = kStgRows * qvae::kBoxW * qvae::kStgPixelBytes
 uint32_t smem_needed(const Tiling& t) {
   const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 2 * 8 * qvae::kMaxStgSlots + 8;
   return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + (t.fuse ? t.SS * kStgSlotBytes : 0u) +
-         (t.overlap ? qvae::kOvlBytes : 0u) +
          qvae::kEpiWarps * t.epi_bufs * qvae::kEpiBufBytes +
          bars +
          16 + 16 + 2 * t.NT * 4;
@@ -184,11 +182,9 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   return (waves * per_tile + tail) * (t.pair ? 1.0 : 1.3);
 }
 
-int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse,
-                  bool overlap) {
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse) {
   if (G != 1 && !(G == 3 && MS <= 2)) return QVAE_ERR_ARG;  // kernel instantiations
   t->fuse = fuse;
-  t->overlap = overlap;
   t->pair = pair;
   t->MS = MS;
   t->NT = NT;
@@ -223,7 +219,7 @@ int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms
   return QVAE_OK;
 }
 
-int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false, bool overlap = false) {
+int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false) {
   bool found = false;
   for (int mode = 1; mode <= 2; ++mode) {
     if (g_force[4] && mode != g_force[4]) continue;
@@ -235,7 +231,7 @@ int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false
         for (int g = 1; g <= 3; g += 2) {
           if (g_force[5] && g != g_force[5]) continue;
           Tiling u;
-          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u, fuse, overlap) != QVAE_OK) continue;
+          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u, fuse) != QVAE_OK) continue;
           u.est_cycles = estimate_cycles(s, u, sms);
           if (!found || u.est_cycles < t->est_cycles) {
             *t = u;
@@ -331,15 +327,10 @@ struct OverlapQuant {
 };
 
 // Row bands of the overlapped variant: at most kMaxBands bands of whole input
-// rows (n, t, h flattened), at least kBandRows rows each, each split into
-// units of kUnitGroups 16-value groups; the last unit of a band may be short,
-// and the last band's surplus units are empty but still counted, so every
-// band completes at band_units.  A producer checks each band once, with one
-// acquire (an L2 round trip), before the first box that reads it: bands as
-// tall as a tile keep that to one or two checks per row of tiles (single-row
-// bands made the checks, not the quantisation, the limit).
+// rows (n, t, h flattened), each split into units of kUnitGroups 16-value
+// groups; the last unit of a band may be short, and the last band's surplus
+// units are empty but still counted, so every band completes at band_units.
 constexpr int kMaxBands = 4095;
-constexpr int kBandRows = 16;
 struct Bands {
   int rows, nbands;
   int64_t groups, total_groups;
@@ -348,7 +339,7 @@ struct Bands {
 int make_bands(const qvae_shape& s, Bands* b) {
   const int64_t R = s.N * s.T * s.H;
   const int64_t per_row = s.W * static_cast<int64_t>(s.Cin) / 16;  // Cin % 32 == 0
-  b->rows = static_cast<int>(std::max<int64_t>(kBandRows, ceil_div(R, kMaxBands)));
+  b->rows = static_cast<int>(std::max<int64_t>(1, ceil_div(R, kMaxBands)));
   b->nbands = static_cast<int>(ceil_div(R, b->rows));
   b->groups = b->rows * per_row;
   b->total_groups = R * per_row;
@@ -396,7 +387,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   qvae_shape sb = s;  // the geometry in bytes: bf16 is tiled as twice the channels of codes
   sb.Cin = s.Cin * elt;
   Tiling t;
-  rc = make_tiling(sb, &t, sms, fuse, oq != nullptr);
+  rc = make_tiling(sb, &t, sms, fuse);
   if (rc) return rc;
   const int nchunks = (sb.Cin + 127) / 128;  // 128-byte channel chunks
 
@@ -670,7 +661,7 @@ int check_layer_args(const qvae_shape* shape, const void* x, const int8_t* xq, v
     return QVAE_ERR_UNSUPPORTED;
   }
   Tiling t;
-  return make_tiling(*shape, &t, *sms_out, false, true);
+  return make_tiling(*shape, &t, *sms_out);
 }
 
 // Pass 1 of the overlapped layer: partial maxima into the workspace, band
@@ -1067,8 +1058,7 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       qvae_shape sb = layers[i].shape;
       if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
-      const bool q8 = layers[i].quantized != 0;
-      if ((rc = make_tiling(sb, &t, sms, q8 && g_fused_quant, q8 && !g_fused_quant))) return rc;
+      if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0 && g_fused_quant))) return rc;
       Bands bd;
       if (layers[i].quantized && (rc = make_bands(layers[i].shape, &bd))) return rc;
       if (layers[i].quantized && act_grid(pixels(layers[i].shape) * layers[i].shape.Cin, sms) * sizeof(uint32_t) >
@@ -1212,7 +1202,7 @@ int qvae_set_conv_cta_limit(int32_t max_ctas) {
 }
 
 int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8) {
-  if (!out8 || variant < 0 || variant > 3) return QVAE_ERR_ARG;
+  if (!out8 || variant < 0 || variant > 2) return QVAE_ERR_ARG;
   int rc = check_shape(shape);
   if (rc) return rc;
   int sms = 148, dev;
@@ -1221,7 +1211,7 @@ int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8
   qvae_shape sb = *shape;
   if (variant == 2) sb.Cin *= 2;  // native precision: tiled by bytes
   Tiling t;
-  if ((rc = make_tiling(sb, &t, sms, variant == 1, variant == 3))) return rc;
+  if ((rc = make_tiling(sb, &t, sms, variant == 1))) return rc;
   out8[0] = t.MS;
   out8[1] = t.NT;
   out8[2] = t.SA;
