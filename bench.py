@@ -3,12 +3,9 @@
 One step = the whole per-call path of every layer of the workload: for each
 layer the activation absmax + INT8 quantisation, then the implicit-GEMM
 convolution with its fused epilogue (weights are quantised and packed once,
-before timing, as a model load would).  By default a layer is the overlapped
-form (qvae_layer_w8a8): the absmax pass, then the convolution whose own extra
-warps write the codes band by band while it runs.  --two-pass times the
-quantise pass and the convolution one after the other; --fused the
-convolution that quantises its bf16 input into shared memory per tile.
-Default workload: the six decoder
+before timing, as a model load would).  --fused times the other form of a
+layer: the absmax pass, then the convolution that quantises its bf16 input
+itself.  Default workload: the six decoder
 layer shapes of a 1024x1024 decode (384->384 @128x128 and @256x256, 384->192
 and 192->192 @512x512, 192->96 and 96->96 @1024x1024, 1% outliers at +-8);
 its first layer is the same tensors as the single decoder top-stage layer
@@ -77,8 +74,6 @@ def parse():
                     help="time the native-precision (bf16 kind::f16) convolution of the workload's layers")
     ap.add_argument("--fused", action="store_true",
                     help="layers as absmax + the convolution quantising its bf16 input in the kernel")
-    ap.add_argument("--two-pass", action="store_true",
-                    help="layers as absmax + quantise passes, then the convolution of the codes")
     ap.add_argument("--chain", default="",
                     help="comma-separated consecutive layers of the workload run as one qvae_decode_layers "
                          "chain, each output feeding the next input (one GPU)")
@@ -362,8 +357,6 @@ class LayerJob:
         self.starts = list(range(0, s.T, self.chunk)) if self.chunk else [0]
         self.dev = dev
         self.fused = bool(args.fused) and not (self.chunk or self.nb)
-        # the overlapped layer: absmax pass, then the convolution that quantises beside the tensor cores
-        self.overlap = not (self.fused or self.chunk or self.nb or args.two_pass)
 
     def set_bytes(self):
         s = self.s
@@ -375,8 +368,8 @@ class LayerJob:
         st = dict(x=self.layer.x.to(dev), xq=torch.empty(self.layer.x.shape, dtype=torch.int8, device=dev),
                   x_scale=torch.empty(1, dtype=torch.float32, device=dev),
                   amax=torch.empty(1, dtype=torch.int32, device=dev),
-                  ws=torch.empty(max(qvae.qvae_act_workspace_bytes(self.layer.x.numel()),
-                                     qvae.qvae_layer_workspace_bytes()), dtype=torch.uint8, device=dev),
+                  ws=torch.empty(qvae.qvae_act_workspace_bytes(self.layer.x.numel()), dtype=torch.uint8,
+                                 device=dev),
                   out=torch.empty((s.N, s.T, s.H, s.W, s.Cout), dtype=torch.bfloat16, device=dev),
                   packed=self.packed0.clone())
         if self.chunk:
@@ -409,17 +402,13 @@ class LayerJob:
     def launches_per_step(self):
         if self.nb:
             return 1 + 2 * self.nb
-        # fused and overlapped: absmax + convolution
-        return 2 if (self.fused or self.overlap) else 3 * len(self.starts)
+        return 2 if self.fused else 3 * len(self.starts)  # fused: absmax + convolution
 
     def _parts(self, st):
         return st["chunks"] if self.chunk else [st]
 
     def act(self, st):
         q = self.qvae
-        if self.overlap:
-            q.qvae_layer_w8a8_absmax(st["x"], self.s.Cout, st["ws"], self.stream)
-            return
         if self.fused:
             q.qvae_act_absmax(st["x"], st["amax"], self.stream)
             return
@@ -441,10 +430,6 @@ class LayerJob:
 
     def conv(self, st):
         q = self.qvae
-        if self.overlap:
-            q.qvae_layer_w8a8_conv(st["x"], st["xq"], st["x_scale"], st["packed"], self.s_w, self.b, st["out"],
-                                   st["ws"], self.stream)
-            return
         if self.fused:
             q.qvae_causal_conv3d_w8a8_fused(st["x"], st["amax"], st["packed"], self.s_w, self.b, st["out"],
                                             st["x_scale"], self.stream)
@@ -459,10 +444,6 @@ class LayerJob:
 
     def step(self, st):
         q = self.qvae
-        if self.overlap:
-            q.qvae_layer_w8a8(st["x"], st["xq"], st["x_scale"], st["packed"], self.s_w, self.b, st["out"],
-                              st["ws"], self.stream)
-            return
         if self.fused:
             self.act(st)
             self.conv(st)
@@ -613,14 +594,11 @@ def run_ours(args):
     outs = torch.empty((s0.N, s0.T, Hs, Ws, s0.Cout), dtype=torch.bfloat16, device=dev)
     switch_ms = []
     xqs = torch.empty(xs.shape, dtype=torch.int8, device=dev)
-    wss = torch.empty(max(qvae.qvae_act_workspace_bytes(xs.numel()), qvae.qvae_layer_workspace_bytes()),
-                      dtype=torch.uint8, device=dev)
+    wss = torch.empty(qvae.qvae_act_workspace_bytes(xs.numel()), dtype=torch.uint8, device=dev)
     for _ in range(2):                            # first call, then the same call warm
         torch.cuda.synchronize()
         t_sw = time.perf_counter()
-        if jobs[0].overlap:
-            qvae.qvae_layer_w8a8(xs, xqs, scs, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, wss, stream)
-        elif jobs[0].fused:
+        if jobs[0].fused:
             qvae.qvae_act_absmax(xs, ams, stream)
             qvae.qvae_causal_conv3d_w8a8_fused(xs, ams, jobs[0].packed0, jobs[0].s_w, jobs[0].b, outs, scs, stream)
         else:
@@ -692,7 +670,7 @@ def run_ours(args):
         key = args.workload if single and len(wl.layers) == 1 else f"{args.workload}[{idx[li]}]"
         # the committed counters describe one whole-layer launch of the two-pass
         # kernel; the fused kernel, row bands and streamed chunks launch otherwise
-        tr = profiled_traffic(("overlap:" if j.overlap else "") + key) if not (j.fused or j.nb or j.chunk) else None
+        tr = None if (j.fused or j.nb or j.chunk) else profiled_traffic(key)
         traffic.append(tr)
         numel = j.layer.x.numel()
         layer_entries.append({
@@ -700,7 +678,7 @@ def run_ours(args):
             "ms": p["layer"], "act_ms": p["act"], "conv_ms": p["conv"], "conv_ms_median": p["conv_median"],
             "layer_tops": lops / (p["layer"] * 1e-3) / 1e12, "conv_tops": lops / (p["conv"] * 1e-3) / 1e12,
             "conv_frac": lops / (p["conv"] * 1e-3) / 1e12 / peak,
-            "act_gbs": (2 if (j.fused or j.overlap) else 5) * numel / (p["act"] * 1e-3) / 1e9,
+            "act_gbs": (2 if j.fused else 5) * numel / (p["act"] * 1e-3) / 1e9,
             "tiling": qvae.qvae_get_conv_tiling(j.s.N, j.s.T, j.s.H, j.s.W, j.s.Cin, j.s.Cout,
                                                 1 if j.fused else 0),
             "dram_bytes_per_conv_launch": tr})
@@ -717,8 +695,6 @@ def run_ours(args):
                           f"({n_sets * per_set / 2**20:.0f} MiB > 3x the 126 MB L2); no flush in the timed region"),
                    "launch": (("one CUDA graph replay per step (per layer: act absmax, conv quantising in its "
                                "producer)" if jobs[0].fused else
-                               "one CUDA graph replay per step (per layer: act absmax, then the conv whose "
-                               "extra warps write the codes band by band beside the MMAs)" if jobs[0].overlap else
                                "one CUDA graph replay per step (per layer: act absmax, act quantise, conv)")
                               if args.launch == "graph" else "direct launches from Python"),
                    "ops_per_step": ops,
@@ -733,17 +709,13 @@ def run_ours(args):
                           "note": "host wall clock, act + conv of the first layer with a device synchronise"},
         "roofline": {"bound": "tensor", "achieved": conv_tops, "peak": peak, "unit": "TOPS",
                      "kernel_variant": ("conv3d_w8a8_fused_kernel (bf16 in, codes made in shared memory)"
-                                        if jobs[0].fused else
-                                        "conv3d_w8a8_overlap_kernel (bf16 in; codes written to HBM band by "
-                                        "band by its own extra warps and read back by TMA)" if jobs[0].overlap
-                                        else "conv3d_w8a8_kernel (INT8 codes in)"),
+                                        if jobs[0].fused else "conv3d_w8a8_kernel (INT8 codes in)"),
                      "frac": conv_tops / peak, "traffic": traffic_mean,
                      "peak_source": f"{peak_src} bf16 burst {bf16_burst} TFLOP/s x {INT8_PER_BF16} "
                                     "(nominal dense INT8/BF16 ratio)",
                      "int8_cublas_tops": int8_tops,
                      "frac_of_int8_cublas": (conv_tops / int8_tops) if int8_tops else None,
-                     "kernel": ("conv3d_w8a8_fused_kernel" if jobs[0].fused else
-                                "conv3d_w8a8_overlap_kernel" if jobs[0].overlap else "conv3d_w8a8_kernel"),
+                     "kernel": "conv3d_w8a8_fused_kernel" if jobs[0].fused else "conv3d_w8a8_kernel",
                      "kernel_ms_mean": conv_total_max / len(jobs), "launches": conv_launches * len(jobs),
                      "note": ("achieved = the layers' ops over the sum of their convolutions' mean CUDA-event "
                               "times; traffic = mean DRAM bytes per conv launch over the layers")},

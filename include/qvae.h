@@ -187,45 +187,6 @@ int qvae_causal_conv3d_w8a8_acc32(const qvae_shape* shape, const int8_t* xq,
                                   const int8_t* wq_packed, int32_t* acc, void* stream);
 
 /*
- * One whole quantised layer from its bf16 input, with the quantisation running
- * beside the convolution instead of before it:
- *   qvae_layer_w8a8 = qvae_act_absmax_quant(x) -> xq, x_scale, then
- *                     qvae_causal_conv3d_w8a8(xq, x_scale, ...) -> out,
- * with the same codes, scale and outputs bit for bit.  Two kernels: the
- * absmax pass, then a convolution whose two extra warps per CTA write the
- * codes of x into xq in row-band order (units of 4096 codes claimed from a
- * device counter, each counted on its band) while its producer waits for the
- * bands a box reads before loading them.  The quantise pass's reading of x and
- * writing of xq thus overlap the tensor cores' work, and the convolution
- * reads most codes from L2 shortly after they were written.
- *   x_bf16     [N][T][H][W][Cin] bf16 (finite), read twice (absmax, codes).
- *   xq         [N][T][H][W][Cin] INT8, written: the codes of x.
- *   x_scale    device fp32, written: absmax(x) / 127.
- *   wq_packed, w_scale, bias_bf16, out_bf16   as qvae_causal_conv3d_w8a8.
- *   workspace  qvae_layer_workspace_bytes() bytes, 16-byte aligned: the partial
- *              maxima and the band counters (at most 4095 bands).  Calls that
- *              may overlap on the GPU need separate workspaces.
- * Sizes with N*T*H*W == 0 write scale 0 and nothing else.  A band wait that
- * runs out of time is reported by qvae_get_error() (QVAE_ERR_TIMEOUT).
- * qvae_layer_w8a8_absmax + qvae_layer_w8a8_conv are the two kernels as two
- * calls (the convolution must directly follow its absmax pass on the same
- * stream, with the same shape, x and workspace); the _acc32 form writes the
- * raw INT32 accumulators acc [N][T][H][W][Cout] instead of out.
- */
-size_t qvae_layer_workspace_bytes(void);
-int qvae_layer_w8a8(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                    const int8_t* wq_packed, const float* w_scale, const void* bias_bf16, void* out_bf16,
-                    void* workspace, size_t workspace_bytes, void* stream);
-int qvae_layer_w8a8_acc32(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                          const int8_t* wq_packed, int32_t* acc, void* workspace, size_t workspace_bytes,
-                          void* stream);
-int qvae_layer_w8a8_absmax(const qvae_shape* shape, const void* x_bf16, void* workspace, size_t workspace_bytes,
-                           void* stream);
-int qvae_layer_w8a8_conv(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                         const int8_t* wq_packed, const float* w_scale, const void* bias_bf16, void* out_bf16,
-                         void* workspace, size_t workspace_bytes, void* stream);
-
-/*
  * Streamed temporal decode (a video decoded in chunks of frames, as for the
  * Wan VAE the release note names): the same convolution over a chunk of
  * shape->T frames whose input carries, in front of the chunk, the last two
@@ -366,25 +327,23 @@ typedef struct qvae_layer {
 
 /* Workspace bytes qvae_decode_layers needs for these layers under the
  * current qvae_set_fused_quant setting: the last quantised layer's activation
- * scale (fp32 at byte 0) and three maximum words (bytes 64, 128, 192); unless
- * the fused convolution is selected, also qvae_layer_workspace_bytes() and the
- * largest quantised input's codes. */
+ * scale (fp32 at byte 0) and three maximum words (bytes 64, 128, 192); with
+ * the two-pass path also the activation workspace and the largest quantised
+ * input's codes. */
 size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n);
 
 /*
- * In order on one stream, for each quantised layer: qvae_layer_w8a8 (the
- * absmax pass, then the convolution into `out` whose own warps write the codes
- * into the workspace beside its MMAs) (with qvae_set_fused_quant(1): the
- * absmax into a workspace word, then the fused convolution, which quantises x
- * into shared memory itself); for each native layer with
+ * In order on one stream, for each quantised layer: the activation absmax +
+ * quantise passes into the workspace, then the W8A8 convolution into `out`
+ * (with qvae_set_fused_quant(1): the absmax into a workspace word, then the
+ * fused convolution, which quantises x itself); for each native layer with
  * packed bf16 weights: the bf16 convolution into `out`; native layers without
  * weights are skipped.
  * All layers are validated before anything is launched.  When a layer's
  * `out` is the next layer's `x` and the next layer is quantised (same N, T,
  * H, W and Cout == next Cin), the convolution also accumulates the maximum
- * bf16 magnitude it writes and the next layer skips its absmax pass: it runs
- * as the quantise pass from that maximum, then the convolution of the codes
- * (fused: the one convolution).  Codes, scales and outputs are the
+ * bf16 magnitude it writes and the next layer skips its absmax pass: each
+ * quantised layer is then one kernel.  Codes, scales and outputs are the
  * same as layer-by-layer qvae_act_absmax_quant + qvae_causal_conv3d_w8a8.
  */
 int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,

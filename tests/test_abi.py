@@ -101,8 +101,8 @@ def test_decode_layers_validates_everything_first():
     arr[1].shape = qvae.make_shape(1, 1, 8, 8, 48, 64)
     arr[1].wq_packed = None                                # without weights it is skipped: not checked
     need = L.qvae_decode_workspace_bytes(arr, 2)
-    # scale + maximum words, partial maxima and band counters, the codes of the largest quantised input
-    assert need == 256 + qvae.qvae_layer_workspace_bytes() + 8 * 8 * 64
+    # scale + maximum words, partial maxima, the codes of the largest quantised input (8 x 8 x 64)
+    assert need == 256 + qvae.qvae_act_workspace_bytes(1) + 8 * 8 * 64
     qvae.qvae_set_fused_quant(1)
     try:
         assert L.qvae_decode_workspace_bytes(arr, 2) == 256       # the fused path keeps no codes

@@ -113,20 +113,6 @@ struct ConvArgs {
   uint32_t stg_slot_bytes;    // stg_rows x 10 pixels x 128 channels x 2 bytes
   uint32_t* zero_word;        // or null: a word set to zero (for a later layer's maximum)
   float one;                  // 1.0f (an operand the compiler cannot fold; see add_f32x2)
-  // overlapped quantisation (conv3d_w8a8_overlap_kernel): two more warps write
-  // the codes of the bf16 input to the code tensor row band by row band while
-  // the convolution, which reads the codes back through tmap_x, runs
-  const uint4* x_in;          // bf16 input, 16 values per 32 bytes
-  uint4* xq_out;              // its codes, 16 per 16 bytes (the tensor tmap_x describes)
-  const uint32_t* partial;    // the absmax pass's partial maxima of x_in
-  int npartial;
-  uint32_t* band_done;        // per row band: units of its codes written and released
-  uint32_t* next_claim;       // the quantising warps' claim counter
-  int band_rows;              // input rows (n, t, h flattened) per band
-  uint32_t band_units;        // units per band: a band is complete at this count
-  int64_t band_groups;        // 16-value groups per band
-  int64_t total_groups;       // numel / 16
-  uint32_t total_units;       // bands x band_units
 };
 
 constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
@@ -138,11 +124,6 @@ constexpr int kMaxStgSlots = 8;
 constexpr uint32_t kStgPixelBytes = 256;            // 128 bf16 channels of one pixel
 constexpr uint32_t kEpiBufBytes = 2048;    // one epilogue staging buffer: 32 pixels x 64 B
 constexpr int kAccBars = 8;                 // accumulator barriers: buffer x sub-tile
-// Streamed quantisation: a unit is 8 groups of 16 values per lane of a warp
-// (8 KB of bf16 in, 4 KB of codes out); a warp claims kClaimUnits units at a time.
-constexpr int kUnitLaneGroups = 8;
-constexpr int kUnitGroups = 32 * kUnitLaneGroups;
-constexpr uint32_t kClaimUnits = 4;
 
 // Packed fp32 pairs (low word = first value).  RN(a * b); and RN(a + b)
 // computed as fma(a, one, b) with `one` = (1.0, 1.0) from a kernel argument:
@@ -469,17 +450,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
 // swizzled layout, into the activation ring -- the same codes as the
 // activation quantiser, with the scale bf16(amax) / 127 taken from one device
 // word.  The producer then loads weights only.
-//
-// kOverlap (INT8 only): x arrives as bf16 together with the absmax pass's
-// partial maxima.  Two more warps quantise the whole tensor into the code
-// tensor in row-band order -- units of 8 KB claimed from a device-wide
-// counter by the quantising warps of every CTA, each unit counted on its band
-// with a release -- while the producer, before each activation box, waits
-// (acquire) until the bands holding the box's rows are complete.  The codes,
-// the scale and the outputs are those of the two activation passes followed
-// by the plain convolution; the quantisation runs beside the tensor cores
-// instead of before them.
-template <bool kBf16, bool kAcc32, bool kPair, bool kFuse, bool kOverlap = false>
+template <bool kBf16, bool kAcc32, bool kPair, bool kFuse>
 __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w,
                                             const CUtensorMap& tmap_out, const ConvArgs& a) {
   extern __shared__ uint8_t smem_raw[];
@@ -591,19 +562,6 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       return true;
     };
     bool waited = false;
-    // overlapped: bands below band_seen are complete; a box reads input rows
-    // c.h0 - 1 .. c.h0 + 16 * MS of one frame, and the bands are in row order
-    int band_seen = 0;
-    auto wait_bands = [&](const TileCoord& c, int frame) -> bool {
-      const int last_h = max(0, min(a.H - 1, c.h0 + kTileRows * a.MS));
-      const int64_t row = (static_cast<int64_t>(c.n) * a.T + frame) * a.H + last_h;
-      const int target = static_cast<int>(row / a.band_rows);
-      if (target < band_seen) return true;
-      for (; band_seen <= target; ++band_seen)
-        if (!wait_counter(a.band_done + band_seen, a.band_units, abort_flag, limit, kErrTimeoutBand)) return false;
-      fence_proxy_async_global();  // the codes were written with plain stores; TMA reads them
-      return true;
-    };
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
       const int kt_lo = (a.carry || c.t >= 2) ? 0 : 2 - c.t;
@@ -618,7 +576,6 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
           waited = true;
         }
         if (!kFuse) {
-          if (kOverlap && !wait_bands(c, frame)) goto producer_done;
           if (!mbar_wait(a_empty + 8 * as, ap ^ 1, abort_flag, limit, kErrTimeoutProducer)) goto producer_done;
           const uint32_t bar = a_full + 8 * as;
           if (leader) mbar_arrive_expect_tx(bar, a.a_box_bytes * tx_mult);
@@ -696,77 +653,6 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       mbar_wait(drain_bar, 0, &dummy, limit, kErrTimeoutDrain);
     }
     __syncwarp();
-  } else if (kOverlap && warp >= 2 + kEpiWarps) {
-    // ------------------------------------------------ overlapped quantisers
-    // Unit u: band u / band_units, groups [g0, g1) of it (at most 256); lane
-    // l takes groups g0 + l + 32k.  The loads of a unit are issued before the
-    // previous unit is released, so the release's wait for the earlier stores
-    // overlaps them.  Claims go out in unit order, so every band below the
-    // claim frontier belongs to a warp that is running.
-    grid_dependency_wait();  // the partial maxima and the zeroed counters are final
-    uint32_t m = 0;
-    for (int k = lane; k < a.npartial; k += 32) m = max(m, __ldcg(a.partial + k));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const float sa = __fdiv_rn(bf16_bits_to_f32(m) * 1.0f, 127.0f);  // clip ratio 1.0
-    const Quantizer z = make_quantizer(sa);
-    const bool zero_scale = sa == 0.0f;
-    if (blockIdx.x == 0 && warp == 2 + kEpiWarps && lane == 0 && a.x_scale_out) *a.x_scale_out = sa;
-    const uint32_t nclaims = (a.total_units + kClaimUnits - 1) / kClaimUnits;
-    const uint32_t claim_stride = gridDim.x * static_cast<uint32_t>(kCvtWarps);
-    auto unit_range = [&](uint32_t unit, int64_t& g0, int64_t& g1) -> int {
-      const int b = static_cast<int>(unit / a.band_units);
-      g0 = b * a.band_groups + static_cast<int64_t>(unit % a.band_units) * kUnitGroups;
-      g1 = min(min(g0 + kUnitGroups, (b + 1) * a.band_groups), a.total_groups);
-      return b;
-    };
-    auto release = [&](int b) {
-      __syncwarp();  // every lane's stores are ordered before lane 0's release
-      if (lane == 0 && check_bounds(b >= 0 && static_cast<int64_t>(b) * a.band_units < a.total_units))
-        red_release_gpu_add(a.band_done + b, 1u);
-      __syncwarp();
-    };
-    int pend = -1;
-    uint32_t u = 0, u_end = 0;
-    while (true) {
-      if (u == u_end) {
-        uint32_t c = 0;
-        if (lane == 0) c = atomicAdd(a.next_claim, 1u);
-        c = __shfl_sync(0xFFFFFFFFu, c, 0);
-        if (c >= nclaims) break;
-        u = c * kClaimUnits;
-        u_end = min(u + kClaimUnits, a.total_units);
-        if (lane == 0 && c + claim_stride < nclaims) {
-          // bring the claim about one round ahead into L2 for the warp that will take it
-          const uint32_t p0 = (c + claim_stride) * kClaimUnits;
-          const uint32_t p1 = min(p0 + kClaimUnits, a.total_units) - 1;
-          int64_t f0, f1, l0, l1;
-          unit_range(p0, f0, f1);
-          unit_range(p1, l0, l1);
-          if (l1 > f0) prefetch_l2(a.x_in + 2 * f0, static_cast<uint32_t>((l1 - f0) * 32));
-        }
-      }
-      int64_t g0, g1;
-      const int b = unit_range(u, g0, g1);
-      ++u;
-      uint4 va[kUnitLaneGroups], vb[kUnitLaneGroups];
-#pragma unroll
-      for (int k = 0; k < kUnitLaneGroups; ++k) {
-        const int64_t g = g0 + lane + 32 * k;
-        if (g < g1) {
-          va[k] = __ldcs(a.x_in + 2 * g);
-          vb[k] = __ldcs(a.x_in + 2 * g + 1);
-        }
-      }
-      if (pend >= 0) release(pend);
-#pragma unroll
-      for (int k = 0; k < kUnitLaneGroups; ++k) {
-        const int64_t g = g0 + lane + 32 * k;
-        if (g < g1 && check_bounds(g >= 0 && g < a.total_groups)) a.xq_out[g] = quant16_x2(z, zero_scale, va[k], vb[k]);
-      }
-      pend = b;
-    }
-    if (pend >= 0) release(pend);
   } else if (kFuse && warp >= 2 + kEpiWarps) {
     // ----------------------------------------------------------- quantisers
     // The activation boxes of the fused variant, in the MMA's order: each
@@ -948,16 +834,14 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     int scale_co0 = -1;
     uint32_t out_max = 0;  // largest |output| written by this lane (bf16 magnitude bits)
     bool dead = false;  // a wait gave up: keep pace with the other warps' table barriers, do no work
-    float overlap_sa = 0.0f;  // overlapped variant: the activation scale (set after the grid dependency wait)
     // Scale and bias table for output channels co0..co0+NT-1.  Every epilogue
     // warp sees the same tiles, so all of them take part; the first barrier
     // lets the previous tile's slices finish reading the old table.
     auto fill_table = [&](int co0) {
       named_barrier_sync(1, 32 * kEpiWarps);
-      const float sa = kBf16     ? 1.0f
-                       : kFuse   ? __fdiv_rn(bf16_bits_to_f32(__ldcg(a.x_amax) & 0x7FFFu) * 1.0f, 127.0f)
-                       : kOverlap ? overlap_sa
-                                 : *a.x_scale;
+      const float sa = kBf16   ? 1.0f
+                       : kFuse ? __fdiv_rn(bf16_bits_to_f32(__ldcg(a.x_amax) & 0x7FFFu) * 1.0f, 127.0f)
+                               : *a.x_scale;
       for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
         sc[j] = kBf16 ? 1.0f : __fmul_rn(sa, a.w_scale[co0 + j]);
         bi[j] = a.bias ? __bfloat162float(a.bias[co0 + j]) : 0.0f;
@@ -966,14 +850,6 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       named_barrier_sync(1, 32 * kEpiWarps);
     };
     grid_dependency_wait();  // the activation scale is final
-    if (kOverlap && !kAcc32) {
-      // the quantising warps' scale, from the same partial maxima
-      uint32_t m = 0;
-      for (int k = lane; k < a.npartial; k += 32) m = max(m, __ldcg(a.partial + k));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      overlap_sa = __fdiv_rn(bf16_bits_to_f32(m) * 1.0f, 127.0f);
-    }
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
       const TileCoord c = decode_tile<kPair>(a, tile, rank);
       if (!kAcc32 && c.co0 != scale_co0) fill_table(c.co0);  // before the accumulators are ready
@@ -984,8 +860,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
         // in the fused variant the quantising warps share these warps' SM
         // sub-partitions: poll with a back-off instead of spinning
         if (lane == 0)
-          ok = mbar_wait(acc_full + 8 * (accb + s), cp, abort_flag, limit, kErrTimeoutEpilogue,
-                         (kFuse || kOverlap) ? 200u : 0u);
+          ok = mbar_wait(acc_full + 8 * (accb + s), cp, abort_flag, limit, kErrTimeoutEpilogue, kFuse ? 200u : 0u);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) {
           dead = true;
@@ -1147,15 +1022,6 @@ __global__ void __launch_bounds__(kConvThreadsFused, 1)
     conv3d_w8a8_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                              const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
   conv3d_body<false, kAcc32, kPair, true>(tmap_x, tmap_w, tmap_out, a);
-}
-
-// W8A8 convolution whose own extra warps quantise its bf16 input into codes,
-// row band by row band, while it runs (scale from the absmax partial maxima).
-template <bool kAcc32, bool kPair>
-__global__ void __launch_bounds__(kConvThreadsFused, 1)
-    conv3d_w8a8_overlap_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                              const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
-  conv3d_body<false, kAcc32, kPair, false, true>(tmap_x, tmap_w, tmap_out, a);
 }
 
 // Native-precision convolution: bf16 values, fp32 accumulators, + bias.

@@ -98,7 +98,6 @@ enum DeviceError : int {
   kErrTimeoutDrain = 0x104,
   kErrTimeoutConvert = 0x105,
   kErrBounds = 0x106,  // a debug build found a load or store outside its tensor or ring
-  kErrTimeoutBand = 0x107,  // a wait for a row band of streamed activation codes
 };
 
 // Debug builds (-DQVAE_DEBUG_CHECKS) check each TMA load's and store's
@@ -247,45 +246,6 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 
 // Programmatic dependent launch: wait for the preceding grid's results / let
 // the next grid start its prologue.  Both are no-ops without the launch attribute.
-// Order this thread's earlier generic-proxy accesses (an acquire of data that
-// other threads wrote with plain stores) before its later async-proxy (TMA)
-// accesses of global memory.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Add to a device-wide counter with release semantics: everything this thread
-// wrote, and everything it observed (e.g. through a warp barrier) before,
-// becomes visible to a thread that acquires the incremented value.
-__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Wait until *p >= target (acquire).  Returns false when the CTA has been told
-// to abort or when the wait ran past `limit_ns` (the error word records
-// err_code); polls with a back-off that leaves the issue slots to other warps.
-__device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target, volatile int* abort_flag,
-                                             uint64_t limit_ns, int err_code) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    __nanosleep(100);
-    if (ld_acquire_gpu(p) >= target) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort_flag = 1;
-      atomicCAS(&g_qvae_error, 0, err_code);
-      return false;
-    }
-  }
-}
-
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

@@ -105,20 +105,15 @@ constexpr int kQuantUnroll = 4;  // 32-byte (16-value) groups in flight per thre
 // x is 16-byte aligned; nvec = numel / 8 full vectors; block 0 also covers the
 // tail.  Each thread keeps kAbsUnroll loads in flight.  Plain cached loads:
 // the most recently read part of x is still in L2 when pass 2, which walks
-// the tensor backwards, starts.  zero_buf (nullable): zero_n words set to
-// zero for the kernel after this one (the band counters of the overlapped
-// convolution, which reads them only after waiting for this grid).
+// the tensor backwards, starts.
 __global__ void __launch_bounds__(kActThreads) act_absmax_kernel(const uint4* __restrict__ x,
                                                                   int64_t nvec,
                                                                   const uint16_t* __restrict__ xs,
                                                                   int64_t numel,
                                                                   uint32_t* __restrict__ partial,
-                                                                  uint32_t* amax_word,
-                                                                  uint32_t* __restrict__ zero_buf,
-                                                                  int zero_n) {
+                                                                  uint32_t* amax_word) {
   __shared__ uint32_t red[kActThreads / 32];
   grid_dependents_launch();  // the quantiser may start its prologue
-  for (int k = blockIdx.x * kActThreads + threadIdx.x; k < zero_n; k += gridDim.x * kActThreads) zero_buf[k] = 0u;
   uint32_t m[4] = {0u, 0u, 0u, 0u};
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kActThreads;
   int64_t i = static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x;

@@ -34,8 +34,8 @@ std::atomic<int32_t> g_cta_limit{0};    // cap on the conv grid (0 = one CTA per
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
-bool g_conv_attr_set[kMaxDevices][16] = {};
-int g_max_clusters[kMaxDevices][3] = {};  // per device, per kernel family (plain, fused, overlapped)
+bool g_conv_attr_set[kMaxDevices][12] = {};
+int g_max_clusters[kMaxDevices][2] = {};  // per device, per thread count (plain, fused)
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
 
@@ -316,54 +316,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size
 // x_amax != null: the fused W8A8 variant -- xq holds the bf16 input, quantised
 // in the kernel with the scale bf16(*x_amax) / 127; x_scale_out (nullable)
 // receives that scale; zero_word (nullable) is set to zero by the kernel.
-// oq != null: the overlapped variant -- xq is the code tensor the kernel's own
-// quantising warps write from oq->x (bf16) while it runs; see OverlapQuant.
-struct OverlapQuant {
-  const void* x;             // bf16 input
-  const uint32_t* partial;   // the absmax pass's partial maxima (npartial words)
-  int npartial;
-  uint32_t* counters;        // claim counter, then one completion counter per band (zeroed by the absmax pass)
-  float* x_scale_out;        // nullable
-};
-
-// Row bands of the overlapped variant: at most kMaxBands bands of whole input
-// rows (n, t, h flattened), each split into units of kUnitGroups 16-value
-// groups; the last unit of a band may be short, and the last band's surplus
-// units are empty but still counted, so every band completes at band_units.
-constexpr int kMaxBands = 4095;
-struct Bands {
-  int rows, nbands;
-  int64_t groups, total_groups;
-  uint32_t units, total_units;
-};
-int make_bands(const qvae_shape& s, Bands* b) {
-  const int64_t R = s.N * s.T * s.H;
-  const int64_t per_row = s.W * static_cast<int64_t>(s.Cin) / 16;  // Cin % 32 == 0
-  b->rows = static_cast<int>(std::max<int64_t>(1, ceil_div(R, kMaxBands)));
-  b->nbands = static_cast<int>(ceil_div(R, b->rows));
-  b->groups = b->rows * per_row;
-  b->total_groups = R * per_row;
-  const int64_t units = ceil_div(b->groups, qvae::kUnitGroups);
-  const int64_t total = units * b->nbands;
-  if (units > INT32_MAX || total > INT32_MAX / 2) return QVAE_ERR_SHAPE;
-  b->units = static_cast<uint32_t>(units);
-  b->total_units = static_cast<uint32_t>(total);
-  return QVAE_OK;
-}
-
 int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
                 const void* wq, const float* w_scale, const void* bias, void* out, void* acc,
                 cudaStream_t stream, bool carry = false, uint32_t* out_amax = nullptr, int halo_top = 0,
                 int halo_bot = 0, bool bf16 = false, const uint32_t* x_amax = nullptr,
-                float* x_scale_out = nullptr, uint32_t* zero_word = nullptr, const OverlapQuant* oq = nullptr) {
+                float* x_scale_out = nullptr, uint32_t* zero_word = nullptr) {
   int rc = check_shape(shape);
   if (rc) return rc;
   const bool fuse = x_amax != nullptr;
   if (fuse && bf16) return QVAE_ERR_ARG;
-  if (oq && (fuse || bf16 || carry || halo_top || halo_bot || !oq->x || !oq->partial || !oq->counters ||
-             oq->npartial <= 0))
-    return QVAE_ERR_ARG;
-  if (oq && (!aligned16(oq->x) || !aligned16(oq->counters))) return QVAE_ERR_ALIGN;
   const int elt = bf16 ? 2 : 1;            // bytes per operand element in shared memory
   const int x_elt = (bf16 || fuse) ? 2 : 1;  // bytes per input element in global memory
   if (halo_top < 0 || halo_top > 1 || halo_bot < 0 || halo_bot > 1) return QVAE_ERR_ARG;
@@ -374,7 +335,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   const bool acc_mode = acc != nullptr;
   const qvae_shape& s = *shape;
   if (pixels(s) == 0) return QVAE_OK;  // nothing to read or write
-  if (!xq || !wq || (!acc_mode && !out) || (!acc_mode && !bf16 && ((!x_scale && !fuse && !oq) || !w_scale)))
+  if (!xq || !wq || (!acc_mode && !out) || (!acc_mode && !bf16 && ((!x_scale && !fuse) || !w_scale)))
     return QVAE_ERR_ARG;
   if (!aligned16(xq) || !aligned16(wq) || (out && !aligned16(out)) || (acc && !aligned16(acc)))
     return QVAE_ERR_ALIGN;
@@ -483,46 +444,17 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   a.stg_rows = kStgRows;
   a.stg_groups = (t.MS * qvae::kTileRows + 2) / kStgRows;
   a.stg_slot_bytes = kStgSlotBytes;
-  a.x_in = nullptr;
-  a.xq_out = nullptr;
-  a.partial = nullptr;
-  a.npartial = 0;
-  a.band_done = nullptr;
-  a.next_claim = nullptr;
-  a.band_rows = 1;
-  a.band_units = 0;
-  a.band_groups = 0;
-  a.total_groups = 0;
-  a.total_units = 0;
-  if (oq) {
-    Bands bd;
-    if ((rc = make_bands(s, &bd))) return rc;
-    a.x_in = static_cast<const uint4*>(oq->x);
-    a.xq_out = reinterpret_cast<uint4*>(const_cast<void*>(xq));
-    a.partial = oq->partial;
-    a.npartial = oq->npartial;
-    a.next_claim = oq->counters;
-    a.band_done = oq->counters + 1;
-    a.band_rows = bd.rows;
-    a.band_units = bd.units;
-    a.band_groups = bd.groups;
-    a.total_groups = bd.total_groups;
-    a.total_units = bd.total_units;
-    a.x_scale_out = oq->x_scale_out;
-  }
 
-  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0) + (fuse ? 8 : 0) + (oq ? 12 : 0);
+  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0) + (fuse ? 8 : 0);
   using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, qvae::ConvArgs);
-  const Kernel kernels[16] = {
-      qvae::conv3d_w8a8_kernel<false, false>,        qvae::conv3d_w8a8_kernel<true, false>,
-      qvae::conv3d_w8a8_kernel<false, true>,         qvae::conv3d_w8a8_kernel<true, true>,
-      qvae::conv3d_bf16_kernel<false, false>,        qvae::conv3d_bf16_kernel<true, false>,
-      qvae::conv3d_bf16_kernel<false, true>,         qvae::conv3d_bf16_kernel<true, true>,
-      qvae::conv3d_w8a8_fused_kernel<false, false>,  qvae::conv3d_w8a8_fused_kernel<true, false>,
-      qvae::conv3d_w8a8_fused_kernel<false, true>,   qvae::conv3d_w8a8_fused_kernel<true, true>,
-      qvae::conv3d_w8a8_overlap_kernel<false, false>, qvae::conv3d_w8a8_overlap_kernel<true, false>,
-      qvae::conv3d_w8a8_overlap_kernel<false, true>,  qvae::conv3d_w8a8_overlap_kernel<true, true>};
-  const int threads = (fuse || oq) ? qvae::kConvThreadsFused : qvae::kConvThreads;
+  const Kernel kernels[12] = {
+      qvae::conv3d_w8a8_kernel<false, false>,       qvae::conv3d_w8a8_kernel<true, false>,
+      qvae::conv3d_w8a8_kernel<false, true>,        qvae::conv3d_w8a8_kernel<true, true>,
+      qvae::conv3d_bf16_kernel<false, false>,       qvae::conv3d_bf16_kernel<true, false>,
+      qvae::conv3d_bf16_kernel<false, true>,        qvae::conv3d_bf16_kernel<true, true>,
+      qvae::conv3d_w8a8_fused_kernel<false, false>, qvae::conv3d_w8a8_fused_kernel<true, false>,
+      qvae::conv3d_w8a8_fused_kernel<false, true>,  qvae::conv3d_w8a8_fused_kernel<true, true>};
+  const int threads = fuse ? qvae::kConvThreadsFused : qvae::kConvThreads;
   const Kernel kernel = kernels[kidx];
   if (!g_conv_attr_set[dev][kidx]) {
     QVAE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
@@ -530,7 +462,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   }
   int grid;
   if (t.pair) {
-    int& max_clusters = g_max_clusters[dev][fuse ? 1 : (oq ? 2 : 0)];
+    int& max_clusters = g_max_clusters[dev][fuse ? 1 : 0];
     if (max_clusters == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * sms);
@@ -605,7 +537,7 @@ int launch_act(const void* x, int64_t numel, int8_t* xq, float* x_scale, void* w
   }
   uint32_t* partial = static_cast<uint32_t*>(ws);
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial, nullptr, nullptr, 0);
+      static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel, partial, nullptr);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
   const int g2 = quant_grid(numel, sms);
@@ -636,59 +568,6 @@ int launch_quant_from_amax(const void* x, int64_t numel, const uint32_t* amax, i
       reinterpret_cast<uint4*>(xq), xq, x_scale, zero_word);
   QVAE_CUDA(cudaGetLastError());
   return QVAE_OK;
-}
-
-// Workspace of the overlapped layer: the absmax pass's partial maxima (4096
-// slots), then the claim counter and one completion counter per row band.
-constexpr size_t kLayerWorkspace = kActWorkspace + 4 * (1 + kMaxBands);
-
-// codes: xq is an argument of the call (the absmax pass alone takes none).
-int check_layer_args(const qvae_shape* shape, const void* x, const int8_t* xq, void* ws, size_t ws_bytes,
-                     Bands* bd, int* sms_out, bool codes = true) {
-  int rc = check_shape(shape);
-  if (rc) return rc;
-  if (!ws || ws_bytes < kLayerWorkspace) return QVAE_ERR_ARG;
-  if (!aligned16(ws)) return QVAE_ERR_ALIGN;
-  if (pixels(*shape) == 0) return QVAE_OK;
-  if (!x || (codes && !xq)) return QVAE_ERR_ARG;
-  if (!aligned16(x) || (codes && !aligned16(xq))) return QVAE_ERR_ALIGN;
-  if ((rc = make_bands(*shape, bd))) return rc;
-  int dev;
-  if ((rc = current_device(&dev))) return rc;
-  if ((rc = sm_count(dev, sms_out))) return rc;
-  if (act_grid(pixels(*shape) * shape->Cin, *sms_out) * sizeof(uint32_t) > kActWorkspace) {
-    t_last_error = "the layer workspace holds fewer partial maxima than this GPU's absmax pass writes";
-    return QVAE_ERR_UNSUPPORTED;
-  }
-  Tiling t;
-  return make_tiling(*shape, &t, *sms_out);
-}
-
-// Pass 1 of the overlapped layer: partial maxima into the workspace, band
-// counters zeroed.
-int launch_layer_absmax(const qvae_shape* shape, const void* x, void* ws, const Bands& bd, int sms,
-                        cudaStream_t st) {
-  const int64_t numel = pixels(*shape) * shape->Cin;
-  const int g1 = act_grid(numel, sms);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kActWorkspace);
-  qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, st>>>(
-      static_cast<const uint4*>(x), numel / 8, static_cast<const uint16_t*>(x), numel,
-      static_cast<uint32_t*>(ws), nullptr, counters, 1 + bd.nbands);
-  QVAE_CUDA(cudaGetLastError());
-  return QVAE_OK;
-}
-
-int launch_layer_conv(const qvae_shape* shape, const void* x, int8_t* xq, float* x_scale, const void* wq,
-                      const float* w_scale, const void* bias, void* out, void* acc, void* ws, int sms,
-                      cudaStream_t st, uint32_t* out_amax = nullptr) {
-  OverlapQuant oq;
-  oq.x = x;
-  oq.partial = static_cast<const uint32_t*>(ws);
-  oq.npartial = act_grid(pixels(*shape) * shape->Cin, sms);
-  oq.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kActWorkspace);
-  oq.x_scale_out = x_scale;
-  return launch_conv(shape, xq, nullptr, wq, w_scale, bias, out, acc, st, false, out_amax, 0, 0, false, nullptr,
-                     nullptr, nullptr, &oq);
 }
 
 }  // namespace
@@ -779,72 +658,6 @@ int qvae_act_absmax_quant(const void* x_bf16, int64_t numel, int8_t* xq, float* 
                     static_cast<cudaStream_t>(stream));
 }
 
-size_t qvae_layer_workspace_bytes(void) { return kLayerWorkspace; }
-
-int qvae_layer_w8a8_absmax(const qvae_shape* shape, const void* x_bf16, void* workspace, size_t workspace_bytes,
-                           void* stream) {
-  Bands bd;
-  int sms = 0, rc;
-  if ((rc = check_layer_args(shape, x_bf16, nullptr, workspace, workspace_bytes, &bd, &sms, false))) return rc;
-  if (pixels(*shape) == 0) return QVAE_OK;
-  return launch_layer_absmax(shape, x_bf16, workspace, bd, sms, static_cast<cudaStream_t>(stream));
-}
-
-int qvae_layer_w8a8_conv(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                         const int8_t* wq_packed, const float* w_scale, const void* bias_bf16, void* out_bf16,
-                         void* workspace, size_t workspace_bytes, void* stream) {
-  Bands bd;
-  int sms = 0, rc;
-  if (!x_scale) return QVAE_ERR_ARG;
-  if ((rc = check_layer_args(shape, x_bf16, xq, workspace, workspace_bytes, &bd, &sms))) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (pixels(*shape) == 0) {
-    QVAE_CUDA(cudaMemsetAsync(x_scale, 0, sizeof(float), st));
-    return QVAE_OK;
-  }
-  if (!wq_packed || !w_scale || !out_bf16) return QVAE_ERR_ARG;
-  return launch_layer_conv(shape, x_bf16, xq, x_scale, wq_packed, w_scale, bias_bf16, out_bf16, nullptr, workspace,
-                           sms, st);
-}
-
-int qvae_layer_w8a8(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                    const int8_t* wq_packed, const float* w_scale, const void* bias_bf16, void* out_bf16,
-                    void* workspace, size_t workspace_bytes, void* stream) {
-  Bands bd;
-  int sms = 0, rc;
-  if (!x_scale) return QVAE_ERR_ARG;
-  if ((rc = check_layer_args(shape, x_bf16, xq, workspace, workspace_bytes, &bd, &sms))) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (pixels(*shape) == 0) {
-    QVAE_CUDA(cudaMemsetAsync(x_scale, 0, sizeof(float), st));
-    return QVAE_OK;
-  }
-  if (!wq_packed || !w_scale || !out_bf16) return QVAE_ERR_ARG;
-  if (!aligned16(wq_packed) || !aligned16(out_bf16)) return QVAE_ERR_ALIGN;
-  if ((rc = launch_layer_absmax(shape, x_bf16, workspace, bd, sms, st))) return rc;
-  return launch_layer_conv(shape, x_bf16, xq, x_scale, wq_packed, w_scale, bias_bf16, out_bf16, nullptr, workspace,
-                           sms, st);
-}
-
-int qvae_layer_w8a8_acc32(const qvae_shape* shape, const void* x_bf16, int8_t* xq, float* x_scale,
-                          const int8_t* wq_packed, int32_t* acc, void* workspace, size_t workspace_bytes,
-                          void* stream) {
-  Bands bd;
-  int sms = 0, rc;
-  if (!x_scale || !acc) return QVAE_ERR_ARG;
-  if ((rc = check_layer_args(shape, x_bf16, xq, workspace, workspace_bytes, &bd, &sms))) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (pixels(*shape) == 0) {
-    QVAE_CUDA(cudaMemsetAsync(x_scale, 0, sizeof(float), st));
-    return QVAE_OK;
-  }
-  if (!wq_packed) return QVAE_ERR_ARG;
-  if (!aligned16(wq_packed) || !aligned16(acc)) return QVAE_ERR_ALIGN;
-  if ((rc = launch_layer_absmax(shape, x_bf16, workspace, bd, sms, st))) return rc;
-  return launch_layer_conv(shape, x_bf16, xq, x_scale, wq_packed, nullptr, nullptr, nullptr, acc, workspace, sms,
-                           st);
-}
-
 int qvae_causal_conv3d_w8a8(const qvae_shape* shape, const int8_t* xq, const float* x_scale,
                             const int8_t* wq_packed, const float* w_scale, const void* bias_bf16,
                             void* out_bf16, void* stream) {
@@ -871,7 +684,7 @@ int qvae_act_absmax(const void* x_bf16, int64_t numel, uint32_t* amax, void* str
   if ((rc = sm_count(dev, &sms))) return rc;
   qvae::act_absmax_kernel<<<act_grid(numel, sms), qvae::kActThreads, 0, st>>>(
       static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, nullptr,
-      amax, nullptr, 0);
+      amax);
   QVAE_CUDA(cudaGetLastError());
   return QVAE_OK;
 }
@@ -990,7 +803,7 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
   // written by the first in this call, so nothing needs clearing.
   qvae::act_absmax_kernel<<<g1, qvae::kActThreads, 0, st>>>(
       static_cast<const uint4*>(x_bf16), numel / 8, static_cast<const uint16_t*>(x_bf16), numel, partial,
-      nullptr, nullptr, 0);
+      nullptr);
   QVAE_CUDA(cudaGetLastError());
   const int64_t nvec2 = numel / 16;
   const int g2 = quant_grid(numel, sms);
@@ -1003,9 +816,9 @@ int qvae_act_absmax_quant_noalloc(const void* x_bf16, int64_t numel, int8_t* xq,
 
 // Workspace of qvae_decode_layers: the activation scale of the last quantised
 // layer (fp32 at byte 0) and three 32-bit maximum words (bytes 64, 128, 192);
-// then, when quantised layers run on codes (not the fused convolution), the
-// overlapped layer's workspace (partial maxima and band counters) and the
-// largest quantised input's codes.
+// then, when quantised layers run as the quantise pass + the convolution of
+// codes, the activation workspace (partial maxima) and the largest quantised
+// input's codes.
 constexpr size_t kDecodeHeader = 256;
 
 std::atomic<bool> g_fused_quant{false};  // quantised layers of qvae_decode_layers: fused convolution
@@ -1016,7 +829,7 @@ size_t qvae_decode_workspace_bytes(const qvae_layer* layers, int32_t n) {
   int64_t max_in = 0;
   for (int32_t i = 0; i < n; ++i)
     if (layers[i].quantized) max_in = std::max<int64_t>(max_in, pixels(layers[i].shape) * layers[i].shape.Cin);
-  return kDecodeHeader + kLayerWorkspace + static_cast<size_t>((max_in + 255) / 256 * 256);
+  return kDecodeHeader + kActWorkspace + static_cast<size_t>((max_in + 255) / 256 * 256);
 }
 
 // The library runs a layer when it is quantised, or when it is a native-
@@ -1047,10 +860,9 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
   const size_t need = qvae_decode_workspace_bytes(layers, n);
   if (!workspace || workspace_bytes < need) return QVAE_ERR_ARG;
   if (!aligned16(workspace)) return QVAE_ERR_ALIGN;
-  int sms = 0;
   if (n > 0) {
-    // every shape has a valid tiling (and row bands) on this GPU before anything is launched
-    int dev = 0, rc = current_device(&dev);
+    // every shape has a valid tiling on this GPU before anything is launched
+    int dev = 0, sms = 0, rc = current_device(&dev);
     if (rc) return rc;
     if ((rc = sm_count(dev, &sms))) return rc;
     for (int32_t i = 0; i < n; ++i) {
@@ -1059,20 +871,13 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
       if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0 && g_fused_quant))) return rc;
-      Bands bd;
-      if (layers[i].quantized && (rc = make_bands(layers[i].shape, &bd))) return rc;
-      if (layers[i].quantized && act_grid(pixels(layers[i].shape) * layers[i].shape.Cin, sms) * sizeof(uint32_t) >
-                                     kActWorkspace) {
-        t_last_error = "the workspace holds fewer partial maxima than this GPU's absmax pass writes";
-        return QVAE_ERR_UNSUPPORTED;
-      }
     }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* x_scale = reinterpret_cast<float*>(ws);
   const bool fused = g_fused_quant.load();
-  void* layer_ws = ws + kDecodeHeader;  // partial maxima, then the band counters
-  int8_t* xq = reinterpret_cast<int8_t*>(ws + kDecodeHeader + kLayerWorkspace);
+  void* partial = ws + kDecodeHeader;
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + kDecodeHeader + kActWorkspace);
   // Layer i reads its input maximum from word i % 3, accumulates its output's
   // maximum (when that output feeds the next quantised layer) into word
   // (i + 1) % 3, and a fused convolution clears word (i + 2) % 3: the word
@@ -1109,20 +914,13 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
         rc = launch_conv(&L.shape, L.x, nullptr, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
                          out_word, 0, 0, false, in_word, x_scale, word[(i + 2) % 3]);
         next_cleared = true;
-      } else if (fed) {
-        // the quantise pass from the accumulated maximum (it also clears out_word), then the convolution
-        if ((rc = launch_quant_from_amax(L.x, numel, in_word, xq, x_scale, out_word, st))) return rc;
+      } else {
+        // quantise pass (which also clears out_word), then the convolution of the codes
+        rc = fed ? launch_quant_from_amax(L.x, numel, in_word, xq, x_scale, out_word, st)
+                 : launch_act(L.x, numel, xq, x_scale, partial, kActWorkspace, st, out_word);
+        if (rc) return rc;
         rc = launch_conv(&L.shape, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr, st, false,
                          out_word);
-        next_cleared = false;
-      } else {
-        // the overlapped layer: the absmax pass, then the convolution whose own warps write the codes
-        if (out_word && !next_cleared) QVAE_CUDA(cudaMemsetAsync(out_word, 0, sizeof(uint32_t), st));
-        Bands bd;
-        if ((rc = make_bands(L.shape, &bd))) return rc;
-        if ((rc = launch_layer_absmax(&L.shape, L.x, layer_ws, bd, sms, st))) return rc;
-        rc = launch_layer_conv(&L.shape, L.x, xq, x_scale, L.wq_packed, L.w_scale, L.bias, L.out, nullptr,
-                               layer_ws, sms, st, out_word);
         next_cleared = false;
       }
     }

@@ -36,8 +36,6 @@ EXPORTS = (
     "qvae_packed_weight_bytes_bf16", "qvae_pack_weights_bf16", "qvae_causal_conv3d_bf16",
     "qvae_causal_conv3d_bf16_acc32", "qvae_causal_conv3d_w8a8_fused", "qvae_causal_conv3d_w8a8_fused_acc32",
     "qvae_set_fused_quant",
-    "qvae_layer_workspace_bytes", "qvae_layer_w8a8_absmax", "qvae_layer_w8a8_conv", "qvae_layer_w8a8",
-    "qvae_layer_w8a8_acc32",
 )
 
 
@@ -94,11 +92,6 @@ def lib():
             "qvae_causal_conv3d_bf16_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_fused": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p, p], ctypes.c_int),
             "qvae_causal_conv3d_w8a8_fused_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p, p], ctypes.c_int),
-            "qvae_layer_workspace_bytes": ([], sz),
-            "qvae_layer_w8a8_absmax": ([ctypes.POINTER(qvae_shape), p, p, sz, p], ctypes.c_int),
-            "qvae_layer_w8a8_conv": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p, p, sz, p], ctypes.c_int),
-            "qvae_layer_w8a8": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, p, p, sz, p], ctypes.c_int),
-            "qvae_layer_w8a8_acc32": ([ctypes.POINTER(qvae_shape), p, p, p, p, p, p, sz, p], ctypes.c_int),
             "qvae_decode_workspace_bytes": ([ctypes.POINTER(qvae_layer), i32], sz),
             "qvae_decode_layers": ([ctypes.POINTER(qvae_layer), i32, p, sz, p], ctypes.c_int),
             "qvae_get_error": ([p], ctypes.c_int),
@@ -324,7 +317,7 @@ def qvae_causal_conv3d_w8a8_fused_acc32(x: torch.Tensor, x_amax: torch.Tensor, w
                                                      _ptr(acc), _stream(stream)))
 
 
-def layer_w8a8_fused(x, wq_packed, w_scale, bias, Cout: int, stream=None, amax=None, scale=None):
+def layer_w8a8(x, wq_packed, w_scale, bias, Cout: int, stream=None, amax=None, scale=None):
     """One quantised layer the fused way: qvae_act_absmax, then the convolution quantising x itself.
     Returns (out, scale)."""
     if amax is None:
@@ -335,64 +328,6 @@ def layer_w8a8_fused(x, wq_packed, w_scale, bias, Cout: int, stream=None, amax=N
     qvae_act_absmax(x, amax, stream)
     qvae_causal_conv3d_w8a8_fused(x, amax, wq_packed, w_scale, bias, out, scale, stream)
     return out, scale
-
-
-# ----------------------------------- one layer, quantisation beside the convolution
-
-def qvae_layer_workspace_bytes() -> int:
-    return int(lib().qvae_layer_workspace_bytes())
-
-
-def _ws(workspace: torch.Tensor):
-    return _ptr(workspace), workspace.numel() * workspace.element_size()
-
-
-def qvae_layer_w8a8_absmax(x: torch.Tensor, Cout: int, workspace: torch.Tensor, stream=None) -> None:
-    shp = shape_of(x, Cout)
-    _check("qvae_layer_w8a8_absmax",
-           lib().qvae_layer_w8a8_absmax(ctypes.byref(shp), _ptr(x), *_ws(workspace), _stream(stream)))
-
-
-def qvae_layer_w8a8_conv(x: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor, wq_packed: torch.Tensor,
-                         w_scale: torch.Tensor, bias: Optional[torch.Tensor], out: torch.Tensor,
-                         workspace: torch.Tensor, stream=None) -> None:
-    shp = shape_of(x, int(out.shape[-1]))
-    _check("qvae_layer_w8a8_conv",
-           lib().qvae_layer_w8a8_conv(ctypes.byref(shp), _ptr(x), _ptr(xq), _ptr(x_scale), _ptr(wq_packed),
-                                      _ptr(w_scale), _ptr(bias), _ptr(out), *_ws(workspace), _stream(stream)))
-
-
-def qvae_layer_w8a8(x: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor, wq_packed: torch.Tensor,
-                    w_scale: torch.Tensor, bias: Optional[torch.Tensor], out: torch.Tensor,
-                    workspace: torch.Tensor, stream=None) -> None:
-    shp = shape_of(x, int(out.shape[-1]))
-    _check("qvae_layer_w8a8",
-           lib().qvae_layer_w8a8(ctypes.byref(shp), _ptr(x), _ptr(xq), _ptr(x_scale), _ptr(wq_packed),
-                                 _ptr(w_scale), _ptr(bias), _ptr(out), *_ws(workspace), _stream(stream)))
-
-
-def qvae_layer_w8a8_acc32(x: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor, wq_packed: torch.Tensor,
-                          acc: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
-    shp = shape_of(x, int(acc.shape[-1]))
-    _check("qvae_layer_w8a8_acc32",
-           lib().qvae_layer_w8a8_acc32(ctypes.byref(shp), _ptr(x), _ptr(xq), _ptr(x_scale), _ptr(wq_packed),
-                                       _ptr(acc), *_ws(workspace), _stream(stream)))
-
-
-def layer_w8a8(x, wq_packed, w_scale, bias, Cout: int, stream=None, workspace=None, acc32: bool = False):
-    """One quantised layer with its quantisation beside the convolution (qvae_layer_w8a8).
-    Returns (out or INT32 accumulators, codes, scale)."""
-    if workspace is None:
-        workspace = torch.empty(qvae_layer_workspace_bytes(), dtype=torch.uint8, device=x.device)
-    xq = torch.empty(x.shape, dtype=torch.int8, device=x.device)
-    scale = torch.empty(1, dtype=torch.float32, device=x.device)
-    if acc32:
-        acc = torch.empty(tuple(x.shape[:-1]) + (Cout,), dtype=torch.int32, device=x.device)
-        qvae_layer_w8a8_acc32(x, xq, scale, wq_packed, acc, workspace, stream)
-        return acc, xq, scale
-    out = torch.empty(tuple(x.shape[:-1]) + (Cout,), dtype=torch.bfloat16, device=x.device)
-    qvae_layer_w8a8(x, xq, scale, wq_packed, w_scale, bias, out, workspace, stream)
-    return out, xq, scale
 
 
 def conv_acc32(xq, wq_packed, Cout: int, stream=None):
