@@ -115,14 +115,8 @@ struct ConvArgs {
   float one;                  // 1.0f (an operand the compiler cannot fold; see add_f32x2)
 };
 
-// Epilogue warps: 8 (warps 2..9, two per TMEM lane quarter) or, for the W8A8
-// kernel on layers whose tile spends long enough in its MMAs, 7 (warps 2..8:
-// quarter 1 has one warp, 5, so the MMA issuer, warp 1, shares its SM
-// sub-partition with one epilogue warp instead of two).
-constexpr int kEpiWarps = 8;   // the most epilogue warps (shared-memory sizing)
-constexpr int kEpiWarpsSolo = 7;
-constexpr int conv_threads(int epi_warps) { return 32 * (2 + epi_warps); }  // producer, MMA, epilogue warps
-constexpr int kConvThreads = conv_threads(kEpiWarps);
+constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter
+constexpr int kConvThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue warps
 constexpr int kCvtWarps = 2;                        // quantising warps of the fused variant
 constexpr int kConvThreadsFused = kConvThreads + 32 * kCvtWarps;
 constexpr int kMaxStages = 12;
@@ -456,7 +450,7 @@ __device__ __forceinline__ bool mma_issue_loop(const ConvArgs& a, const MmaRings
 // swizzled layout, into the activation ring -- the same codes as the
 // activation quantiser, with the scale bf16(amax) / 127 taken from one device
 // word.  The producer then loads weights only.
-template <bool kBf16, bool kAcc32, bool kPair, bool kFuse, int kEpiW = kEpiWarps>
+template <bool kBf16, bool kAcc32, bool kPair, bool kFuse>
 __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w,
                                             const CUtensorMap& tmap_out, const ConvArgs& a) {
   extern __shared__ uint8_t smem_raw[];
@@ -468,7 +462,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
   const uint32_t b_ring = a_ring + a.SA * a.a_stage_bytes;
   const uint32_t stg_ring = b_ring + a.SB * a.b_stage_bytes;                     // fused: bf16 row groups
   const uint32_t epi_stage = stg_ring + (kFuse ? a.SS * a.stg_slot_bytes : 0u);  // 1024-aligned
-  const uint32_t bars = epi_stage + kEpiW * a.epi_bufs * kEpiBufBytes;  // 8-byte mbarriers
+  const uint32_t bars = epi_stage + kEpiWarps * a.epi_bufs * kEpiBufBytes;  // 8-byte mbarriers
   const uint32_t a_full = bars, a_empty = a_full + 8 * kMaxStages;
   const uint32_t b_full = a_empty + 8 * kMaxStages, b_empty = b_full + 8 * kMaxStages;
   const uint32_t acc_full = b_empty + 8 * kMaxStages, acc_empty = acc_full + 8 * kAccBars;
@@ -511,7 +505,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     }
     for (int i = 0; i < kAccBars; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, kPair ? 2 * kEpiW : kEpiW);  // one arrive per epilogue warp (of both CTAs)
+      mbar_init(acc_empty + 8 * i, kPair ? 2 * kEpiWarps : kEpiWarps);  // one arrive per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -659,7 +653,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
       mbar_wait(drain_bar, 0, &dummy, limit, kErrTimeoutDrain);
     }
     __syncwarp();
-  } else if (kFuse && warp >= 2 + kEpiW) {
+  } else if (kFuse && warp >= 2 + kEpiWarps) {
     // ----------------------------------------------------------- quantisers
     // The activation boxes of the fused variant, in the MMA's order: each
     // box (tile, temporal tap, 128-channel chunk) is 16*MS + 2 rows x 10
@@ -673,7 +667,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     // The warp that finishes a staging slot last refills it with the group SS
     // positions ahead.  When a box is complete each warp fences its shared-
     // memory writes for the tensor cores and arrives on the (leader's) a_full.
-    const int cw = warp - (2 + kEpiW);
+    const int cw = warp - (2 + kEpiWarps);
     const int ct = cw * 32 + lane;
     struct Pos {
       int tile, kb, g, nkb, kt_lo;
@@ -828,11 +822,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     // columns beyond the image edge.  The TMEM load of a warp's next slice is in flight while the
     // current one is converted.
     const int q = warp & 3;
-    // slices of a sub-tile: the two warps of a quarter alternate (step 2);
-    // quarter 1's single warp takes them all (step 1)
-    const bool solo = kEpiW == kEpiWarpsSolo && q == 1;
-    const int half = solo ? 0 : (warp - 2) >> 2;
-    const int jstep = solo ? 1 : 2;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int nsl = a.NT >> 5;
     float* const sc = epi_smem;
@@ -848,16 +838,16 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
     // warp sees the same tiles, so all of them take part; the first barrier
     // lets the previous tile's slices finish reading the old table.
     auto fill_table = [&](int co0) {
-      named_barrier_sync(1, 32 * kEpiW);
+      named_barrier_sync(1, 32 * kEpiWarps);
       const float sa = kBf16   ? 1.0f
                        : kFuse ? __fdiv_rn(bf16_bits_to_f32(__ldcg(a.x_amax) & 0x7FFFu) * 1.0f, 127.0f)
                                : *a.x_scale;
-      for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiW) {
+      for (int j = (warp - 2) * 32 + lane; j < a.NT; j += 32 * kEpiWarps) {
         sc[j] = kBf16 ? 1.0f : __fmul_rn(sa, a.w_scale[co0 + j]);
         bi[j] = a.bias ? __bfloat162float(a.bias[co0 + j]) : 0.0f;
       }
       scale_co0 = co0;
-      named_barrier_sync(1, 32 * kEpiW);
+      named_barrier_sync(1, 32 * kEpiWarps);
     };
     grid_dependency_wait();  // the activation scale is final
     for (int tile = first_tile; tile < a.num_tiles; tile += tile_step) {
@@ -952,7 +942,7 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
               // a box that starts below the last row is clipped whole by the tensor map
               if (check_bounds((c.co0 + cc) % 8 == 0 && c.co0 + cc + 32 <= a.Cout && c.w0 >= 0 && c.w0 < a.W &&
                                c.h0 + s * kTileRows + q * 4 >= 0 && c.t < a.T && c.n < a.N &&
-                               sbuf + kEpiBufBytes <= epi_stage + static_cast<uint32_t>(kEpiW * a.epi_bufs) * kEpiBufBytes))
+                               sbuf + kEpiBufBytes <= epi_stage + static_cast<uint32_t>(kEpiWarps * a.epi_bufs) * kEpiBufBytes))
                 tma_store_5d(&tmap_out, sbuf, c.co0 + cc, c.w0, c.h0 + s * kTileRows + q * 4, c.t, c.n);
               bulk_commit_group();
             }
@@ -960,20 +950,20 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
           }
         };
         uint32_t va[32], vb[32];
-        // this warp's slices of the sub-tile: jj = j0, j0 + jstep, ... (the
-        // two warps of a quarter alternate over the tile's slices in order)
-        int jj = solo ? 0 : (half + s * nsl) & 1;
+        // this warp's slices of the sub-tile: jj = j0, j0 + 2, ... (the two
+        // warps of a quarter alternate over the tile's slices in order)
+        int jj = (half + s * nsl) & 1;
         if (jj < nsl) issue(jj, va);
         while (jj < nsl) {
           tmem_ld_wait(va);
-          if (jj + jstep < nsl) issue(jj + jstep, vb);
+          if (jj + 2 < nsl) issue(jj + 2, vb);
           process(jj, va);
-          jj += jstep;
+          jj += 2;
           if (jj >= nsl) break;
           tmem_ld_wait(vb);
-          if (jj + jstep < nsl) issue(jj + jstep, va);
+          if (jj + 2 < nsl) issue(jj + 2, va);
           process(jj, vb);
-          jj += jstep;
+          jj += 2;
         }
         tc_fence_before();
         __syncwarp();
@@ -1019,11 +1009,11 @@ __device__ __forceinline__ void conv3d_body(const CUtensorMap& tmap_x, const CUt
 }
 
 // W8A8 convolution: INT8 codes, INT32 accumulators, FP32 rescale + bias.
-template <bool kAcc32, bool kPair, int kEpiW>
-__global__ void __launch_bounds__(conv_threads(kEpiW), 1)
+template <bool kAcc32, bool kPair>
+__global__ void __launch_bounds__(kConvThreads, 1)
     conv3d_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_out, const ConvArgs a) {
-  conv3d_body<false, kAcc32, kPair, false, kEpiW>(tmap_x, tmap_w, tmap_out, a);
+  conv3d_body<false, kAcc32, kPair, false>(tmap_x, tmap_w, tmap_out, a);
 }
 
 // W8A8 convolution quantising its bf16 input in the kernel (scale from a maximum word).

@@ -34,8 +34,8 @@ std::atomic<int32_t> g_cta_limit{0};    // cap on the conv grid (0 = one CTA per
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
-bool g_conv_attr_set[kMaxDevices][16] = {};
-int g_max_clusters[kMaxDevices][16] = {};  // per device and kernel
+bool g_conv_attr_set[kMaxDevices][12] = {};
+int g_max_clusters[kMaxDevices][2] = {};  // per device, per thread count (plain, fused)
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per block on sm_100
 
@@ -88,7 +88,6 @@ struct Tiling {
   int MS, NT, SA, SB, acc_stages, G;
   bool split;    // per-sub-tile accumulator hand-off
   int epi_bufs;  // epilogue staging buffers per warp
-  int epi_warps; // epilogue warps: 8, or 7 (quarter 1 served by one warp; W8A8 kernel only)
   bool fuse;     // quantisation in the kernel: a bf16 staging ring of SS row groups
   int SS;
   uint32_t a_stage_bytes, a_box_bytes, b_tap_bytes, b_stage_bytes, tmem_cols, smem_bytes;
@@ -104,7 +103,7 @@ constexpr uint32_t kStgSlotBytes = kStgRows * qvae::kBoxW * qvae::kStgPixelBytes
 uint32_t smem_needed(const Tiling& t) {
   const uint32_t bars = 8 * qvae::kMaxStages * 4 + 2 * 8 * qvae::kAccBars + 2 * 8 * qvae::kMaxStgSlots + 8;
   return 1024 + t.SA * t.a_stage_bytes + t.SB * t.b_stage_bytes + (t.fuse ? t.SS * kStgSlotBytes : 0u) +
-         t.epi_warps * t.epi_bufs * qvae::kEpiBufBytes +
+         qvae::kEpiWarps * t.epi_bufs * qvae::kEpiBufBytes +
          bars +
          16 + 16 + 2 * t.NT * 4;
 }
@@ -183,29 +182,9 @@ double estimate_cycles(const qvae_shape& s, const Tiling& t, int sms) {
   return (waves * per_tile + tail) * (t.pair ? 1.0 : 1.3);
 }
 
-// Cycles one epilogue warp needs per 32-channel slice of a 128-pixel sub-tile
-// (TMEM load, rescale, bf16 pack, staging, TMA store), and how much longer a
-// sub-tile's MMAs must take than quarter 1's single warp needs for all its
-// slices before the seven-warp epilogue is used: the 96 -> 96 layers (nine
-// taps of three k-steps per sub-tile) measured 13 % slower with it, the
-// 192- and 384-channel inputs 5-17 % faster.
-constexpr double kSoloSliceCycles = 300.0;
-constexpr double kSoloMargin = 2.5;
-
-int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse,
-                  bool solo_ok) {
+int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms, Tiling* t, bool fuse) {
   if (G != 1 && !(G == 3 && MS <= 2)) return QVAE_ERR_ARG;  // kernel instantiations
   t->fuse = fuse;
-  t->epi_warps = qvae::kEpiWarps;
-  if (solo_ok && !fuse) {
-    double taps_t = 0;
-    for (int64_t f = 0; f < std::min<int64_t>(s.T, 2); ++f) taps_t += static_cast<double>(f + 1);
-    if (s.T > 2) taps_t += 3.0 * (s.T - 2);
-    taps_t /= std::max<int64_t>(s.T, 1);
-    const double mma = std::max(0.52 * NT + 8.0, 60.0 + 0.17 * NT);  // cycles per MMA, as in estimate_cycles
-    const double mma_subtile = taps_t * 9.0 * (s.Cin / 32.0) * mma;
-    if (mma_subtile >= kSoloMargin * kSoloSliceCycles * (NT / 32)) t->epi_warps = qvae::kEpiWarpsSolo;
-  }
   t->pair = pair;
   t->MS = MS;
   t->NT = NT;
@@ -240,8 +219,7 @@ int make_geometry(const qvae_shape& s, bool pair, int MS, int NT, int G, int sms
   return QVAE_OK;
 }
 
-// solo_ok: the W8A8 convolution of codes (the only kernel built with the seven-warp epilogue).
-int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false, bool solo_ok = false) {
+int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false) {
   bool found = false;
   for (int mode = 1; mode <= 2; ++mode) {
     if (g_force[4] && mode != g_force[4]) continue;
@@ -253,7 +231,7 @@ int make_tiling(const qvae_shape& s, Tiling* t, int sms = 148, bool fuse = false
         for (int g = 1; g <= 3; g += 2) {
           if (g_force[5] && g != g_force[5]) continue;
           Tiling u;
-          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u, fuse, solo_ok) != QVAE_OK) continue;
+          if (make_geometry(s, mode == 2, ms, nt, g, sms, &u, fuse) != QVAE_OK) continue;
           u.est_cycles = estimate_cycles(s, u, sms);
           if (!found || u.est_cycles < t->est_cycles) {
             *t = u;
@@ -370,7 +348,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   qvae_shape sb = s;  // the geometry in bytes: bf16 is tiled as twice the channels of codes
   sb.Cin = s.Cin * elt;
   Tiling t;
-  rc = make_tiling(sb, &t, sms, fuse, !bf16 && !fuse);
+  rc = make_tiling(sb, &t, sms, fuse);
   if (rc) return rc;
   const int nchunks = (sb.Cin + 127) / 128;  // 128-byte channel chunks
 
@@ -467,20 +445,16 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   a.stg_groups = (t.MS * qvae::kTileRows + 2) / kStgRows;
   a.stg_slot_bytes = kStgSlotBytes;
 
-  const bool solo = t.epi_warps == qvae::kEpiWarpsSolo;
-  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (solo ? 12 : (bf16 ? 4 : 0) + (fuse ? 8 : 0));
+  const int kidx = (acc_mode ? 1 : 0) + (t.pair ? 2 : 0) + (bf16 ? 4 : 0) + (fuse ? 8 : 0);
   using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, qvae::ConvArgs);
-  constexpr int E8 = qvae::kEpiWarps, E7 = qvae::kEpiWarpsSolo;
-  const Kernel kernels[16] = {
-      qvae::conv3d_w8a8_kernel<false, false, E8>,   qvae::conv3d_w8a8_kernel<true, false, E8>,
-      qvae::conv3d_w8a8_kernel<false, true, E8>,    qvae::conv3d_w8a8_kernel<true, true, E8>,
+  const Kernel kernels[12] = {
+      qvae::conv3d_w8a8_kernel<false, false>,       qvae::conv3d_w8a8_kernel<true, false>,
+      qvae::conv3d_w8a8_kernel<false, true>,        qvae::conv3d_w8a8_kernel<true, true>,
       qvae::conv3d_bf16_kernel<false, false>,       qvae::conv3d_bf16_kernel<true, false>,
       qvae::conv3d_bf16_kernel<false, true>,        qvae::conv3d_bf16_kernel<true, true>,
       qvae::conv3d_w8a8_fused_kernel<false, false>, qvae::conv3d_w8a8_fused_kernel<true, false>,
-      qvae::conv3d_w8a8_fused_kernel<false, true>,  qvae::conv3d_w8a8_fused_kernel<true, true>,
-      qvae::conv3d_w8a8_kernel<false, false, E7>,   qvae::conv3d_w8a8_kernel<true, false, E7>,
-      qvae::conv3d_w8a8_kernel<false, true, E7>,    qvae::conv3d_w8a8_kernel<true, true, E7>};
-  const int threads = fuse ? qvae::kConvThreadsFused : qvae::conv_threads(t.epi_warps);
+      qvae::conv3d_w8a8_fused_kernel<false, true>,  qvae::conv3d_w8a8_fused_kernel<true, true>};
+  const int threads = fuse ? qvae::kConvThreadsFused : qvae::kConvThreads;
   const Kernel kernel = kernels[kidx];
   if (!g_conv_attr_set[dev][kidx]) {
     QVAE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
@@ -488,7 +462,7 @@ int launch_conv(const qvae_shape* shape, const void* xq, const float* x_scale,
   }
   int grid;
   if (t.pair) {
-    int& max_clusters = g_max_clusters[dev][kidx];
+    int& max_clusters = g_max_clusters[dev][fuse ? 1 : 0];
     if (max_clusters == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * sms);
@@ -896,8 +870,7 @@ int qvae_decode_layers(const qvae_layer* layers, int32_t n, void* workspace,
       qvae_shape sb = layers[i].shape;
       if (!layers[i].quantized) sb.Cin *= 2;  // a native layer is tiled by bytes
       Tiling t;
-      const bool q8 = layers[i].quantized != 0;
-      if ((rc = make_tiling(sb, &t, sms, q8 && g_fused_quant, q8 && !g_fused_quant))) return rc;
+      if ((rc = make_tiling(sb, &t, sms, layers[i].quantized != 0 && g_fused_quant))) return rc;
     }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -1036,7 +1009,7 @@ int qvae_get_conv_tiling(const qvae_shape* shape, int32_t variant, int32_t* out8
   qvae_shape sb = *shape;
   if (variant == 2) sb.Cin *= 2;  // native precision: tiled by bytes
   Tiling t;
-  if ((rc = make_tiling(sb, &t, sms, variant == 1, variant == 0))) return rc;
+  if ((rc = make_tiling(sb, &t, sms, variant == 1))) return rc;
   out8[0] = t.MS;
   out8[1] = t.NT;
   out8[2] = t.SA;
