@@ -216,3 +216,28 @@ def test_native_layer_argument_checks():
     assert conv(ctypes.byref(ok), FAKE, FAKE, None, FAKE_ODD, None) == qvae.QVAE_ERR_ALIGN
     assert conv(ctypes.byref(qvae.make_shape(1, 1, 0, 8, 64, 64)), None, None, None, None, None) == qvae.QVAE_OK
     assert L.qvae_causal_conv3d_bf16_acc32(ctypes.byref(ok), FAKE, FAKE, None, None) == qvae.QVAE_ERR_ARG
+
+
+# Tilings measured best on a B200 for the decoder layer shapes (forced-tiling
+# sweeps with bench-style timing): a change to the cost model that picks
+# another one for these shapes must come with a new measurement.
+MEASURED_BEST = [
+    # (T, H, W, Cin, Cout) -> (mode, MS, NT, G, accumulator buffers)
+    ((1, 128, 128, 384, 384), (2, 1, 192, 3, 2)),
+    ((1, 256, 256, 384, 384), (2, 1, 192, 3, 2)),
+    ((1, 512, 512, 384, 192), (2, 1, 192, 3, 2)),
+    ((1, 512, 512, 192, 192), (2, 1, 192, 3, 2)),
+    ((1, 1024, 1024, 192, 96), (2, 2, 96, 3, 2)),
+    ((1, 1024, 1024, 96, 96), (2, 2, 96, 3, 2)),
+    ((1, 105, 157, 384, 384), (1, 1, 192, 3, 2)),
+    ((1, 420, 628, 384, 192), (2, 1, 192, 3, 2)),
+    ((1, 840, 1256, 96, 96), (2, 2, 96, 3, 2)),
+    ((8, 240, 416, 192, 192), (2, 2, 192, 3, 1)),
+]
+
+
+@pytest.mark.parametrize("shape,want", MEASURED_BEST, ids=[str(s) for s, _ in MEASURED_BEST])
+def test_cost_model_picks_the_measured_best_tiling(shape, want):
+    T, H, W, Cin, Cout = shape
+    t = qvae.qvae_get_conv_tiling(1, T, H, W, Cin, Cout, 0)
+    assert (t["mode"], t["MS"], t["NT"], t["G"], t["acc_buffers"]) == want
